@@ -1,0 +1,179 @@
+/*
+ * kie.h -- C ABI of the batch-1 decode engine (libkie.so), NVIDIA B200 (sm_100a).
+ *
+ * What the library computes. The pages describe a "persistent monokernel": one
+ * GPU-resident program that runs the whole per-token decode step -- MatMul,
+ * attention, normalization and sampling -- and hands each new token back to
+ * itself without returning control to the CPU ("メモリの壁を打破する：標準的なGPUで
+ * 3,000 tokens/sの推論を実現する", section "1. The Monokernel Runtime"; "Kog、より深い
+ * GPU最適化でAI推論を高速化できると賭ける", section "KogがGPU推論の最適化をさらに
+ * 深める理由"). At batch 1 the step is bound by streaming every active weight from
+ * HBM once per token (same first page, section "ボトルネック：計算量ではなくメモリ
+ * 帯域幅"), and launch, host-scheduling and synchronisation overheads are what the
+ * persistent design removes (section "マイクロ秒が失われる場所").
+ *
+ * The model is a pre-norm decoder: RMSNorm, q/k/v projections, RoPE (half-split
+ * pairs), causal attention over an fp16 KV cache, output projection + residual,
+ * RMSNorm, SwiGLU MLP (or routed top-k SwiGLU experts plus a shared expert) +
+ * residual, final RMSNorm, untied LM head and greedy argmax (lowest index on
+ * exact ties). Weights are fp16; activations and accumulation are fp32.
+ *
+ * Conventions common to every call:
+ *  - Every call is synchronous on the given stream: it returns after the work it
+ *    queued has completed. `stream` is a cudaStream_t (NULL = legacy default).
+ *  - One context serves one request on one GPU. Calls on one context are not
+ *    thread-safe; distinct contexts are independent.
+ *  - A device-side failure (a wait that ran past its deadline, a failed device
+ *    check) poisons the context: every call except kie_reset, kie_destroy,
+ *    kie_last_error, kie_position and kie_get_info then returns KIE_ERR_STATE.
+ *  - On any error nothing of the failed call's effect on the context state
+ *    (position, pending token) is kept, except that a poisoned context's KV
+ *    cache contents are undefined until kie_reset.
+ */
+#ifndef KIE_H_
+#define KIE_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct kie_ctx kie_ctx; /* opaque, owned by the library */
+
+typedef enum {
+  KIE_OK = 0,
+  KIE_ERR_INVALID_ARG = -1,  /* bad pointer, size, shape, name or token id        */
+  KIE_ERR_STATE = -2,        /* call out of order (decode before load, poisoned)  */
+  KIE_ERR_CONTEXT_FULL = -3, /* position + tokens would exceed max_ctx            */
+  KIE_ERR_CUDA = -4,         /* a CUDA runtime call failed (message in last_error) */
+  KIE_ERR_TIMEOUT = -5,      /* a device-side wait gave up after its deadline     */
+  KIE_ERR_DEVICE = -6,       /* a device-side check failed                        */
+  KIE_ERR_OOM = -7           /* device or host allocation failed                  */
+} kie_status;
+
+/* Model shape. Dense models set n_experts = top_k = ffn_expert = ffn_shared = 0
+ * and ffn > 0; MoE models set ffn = 0 and the four expert fields.
+ * Constraints: d_model, n_heads*head_dim, ffn, ffn_expert, ffn_shared multiples
+ * of 8; head_dim 64 or 128; each KV head serves 1 to 4 query heads (query
+ * head h reads KV head floor(h * n_kv_heads / n_heads)); max_ctx >= 1. */
+typedef struct {
+  int32_t n_layers, d_model, n_heads, n_kv_heads, head_dim, ffn, vocab;
+  int32_t n_experts, top_k, ffn_expert, ffn_shared;
+  int32_t max_ctx;
+  float rms_eps;    /* RMSNorm: x / sqrt(mean(x^2) + rms_eps) * g            */
+  float rope_theta; /* RoPE angle of pair i at position p: p * theta^(-2i/dh) */
+} kie_config;
+
+/* One weight tensor, fp16, row-major. Matrices are W[out, in] (y = W x):
+ *   embed [V, d]; lm_head [V, d]; final_norm [d]
+ *   layers.{l}.attn_norm [d]; .wq [hq*dh, d]; .wk, .wv [hk*dh, d]; .wo [d, hq*dh]
+ *   layers.{l}.mlp_norm [d]
+ *   dense: layers.{l}.w_gate, .w_up [ffn, d]; .w_down [d, ffn]
+ *   MoE:   layers.{l}.router [E, d];
+ *          layers.{l}.experts.{e}.w_gate, .w_up [ffe, d]; .w_down [d, ffe]
+ *          layers.{l}.shared.w_gate, .w_up [ffs, d]; .w_down [d, ffs]
+ * Vectors give shape {n, 1} or {1, n}. `on_device` = 1 means `data` is a device
+ * pointer on the context's device (16-byte aligned), 0 a host pointer
+ * (pageable or pinned). */
+typedef struct {
+  const char* name;
+  const void* data;
+  int64_t shape[2];
+  int32_t on_device;
+} kie_tensor;
+
+/* Optional per-call controls of kie_decode (pass NULL for defaults). Every
+ * pointer may be host or device memory (detected per call), caller-owned. */
+typedef struct {
+  const int32_t* forced_tokens; /* [n]: token fed back after step i; -1 = argmax.
+                                   Used for teacher forcing; NULL = free run.   */
+  float* logits_out;            /* [n][vocab] fp32 logits of every step; NULL = none */
+  float* margins_out;           /* [n] top-1 minus second-largest logit; NULL = none */
+  uint32_t timeout_ms;          /* deadline of every device-side wait; 0 = 1000 ms    */
+  int32_t fault_cta;            /* test hook: this CTA skips its arrival at grid      */
+  int32_t fault_barrier;        /*   barrier number fault_barrier; -1 = off           */
+  uint64_t* trace_out;          /* device [grid][trace_cap][2] globaltimer stamps of
+                                   each grid barrier's arrival and release; NULL = off */
+  int32_t trace_cap;            /* barriers recorded per CTA                          */
+} kie_decode_opts;
+
+/* Static facts about a loaded context, for measurement. */
+typedef struct {
+  int32_t grid;               /* CTAs of the persistent launch (one per SM)            */
+  int32_t threads;            /* threads per CTA                                      */
+  int32_t n_stages;           /* shared-memory ring stages per CTA                    */
+  int32_t stage_bytes;        /* bytes per ring stage                                 */
+  int32_t smem_bytes;         /* dynamic shared memory per CTA                        */
+  int32_t barriers_per_token; /* grid barriers per decoded token                      */
+  int64_t stream_bytes;       /* weight bytes streamed per decoded token (dense: all
+                                 matrices; MoE: router, shared and top_k experts),
+                                 plus norm gains and one embedding row                */
+  int64_t kv_bytes_per_pos;   /* K+V bytes read per cached position per token         */
+  int64_t resident_bytes;     /* device bytes held by the packed weights              */
+  int64_t launches;           /* kernels this context has launched so far             */
+} kie_info;
+
+/* Create a context on CUDA device `device`. Validates the shape, picks the
+ * launch geometry and allocates the KV cache and scratch (no weights yet).
+ * Errors: INVALID_ARG (shape), CUDA, OOM. On success *out owns the context. */
+kie_status kie_create(const kie_config* cfg, int device, kie_ctx** out);
+
+/* Copy and pack the model weights into library-owned device memory (the
+ * phase-ordered, per-CTA weight tape). The caller keeps ownership of its
+ * buffers and may free them when the call returns. All tensors named in the
+ * kie_tensor comment must be given exactly once with the stated shapes.
+ * May be called again to replace the weights; resets the position.
+ * Errors: INVALID_ARG (missing/extra/misshapen tensor), CUDA, OOM. */
+kie_status kie_load_weights(kie_ctx* ctx, const kie_tensor* tensors, int n_tensors,
+                            void* stream);
+
+/* Append `n` prompt tokens (host array, ids in [0, vocab)). Commits the pending
+ * token (if any) and tokens[0..n-2] to the KV cache; tokens[n-1] becomes the
+ * pending token. No logits are computed. One persistent launch.
+ * Errors: STATE (no weights / poisoned), INVALID_ARG, CONTEXT_FULL, CUDA,
+ * TIMEOUT. */
+kie_status kie_prefill(kie_ctx* ctx, const int32_t* tokens, int n, void* stream);
+
+/* Decode `n_tokens` tokens in ONE persistent launch. Step i forwards the pending
+ * token at the current position, takes the greedy argmax, writes it to
+ * out_tokens[i] (host or device, caller-owned, [n_tokens]) and makes it (or
+ * forced_tokens[i] when >= 0) the pending token for step i+1.
+ * Errors: STATE (no pending token, no weights, poisoned), INVALID_ARG,
+ * CONTEXT_FULL (position + n_tokens > max_ctx; checked before launch), CUDA,
+ * TIMEOUT (context poisoned), DEVICE (context poisoned). */
+kie_status kie_decode(kie_ctx* ctx, int n_tokens, int32_t* out_tokens,
+                      const kie_decode_opts* opts, void* stream);
+
+/* Truncate the sequence to its first `pos` committed positions (0 <= pos <=
+ * current position) and make `pending` (in [0, vocab)) the token fed to the
+ * next forward, e.g. to regenerate from a prefix. KV entries at positions >= pos
+ * are simply overwritten by later calls. Host-side only, no GPU work.
+ * Errors: INVALID_ARG, STATE (no weights, poisoned). */
+kie_status kie_rewind(kie_ctx* ctx, int32_t pos, int32_t pending);
+
+/* Rewind to an empty sequence: position 0, no pending token, error and poison
+ * cleared. Keeps the weights and the KV allocation. */
+kie_status kie_reset(kie_ctx* ctx);
+
+/* Free every resource of the context. NULL is accepted. */
+kie_status kie_destroy(kie_ctx* ctx);
+
+/* Message of the last failed call on this context ("" if none). Valid until the
+ * next call on the same context. NULL ctx gives the last kie_create failure. */
+const char* kie_last_error(const kie_ctx* ctx);
+
+/* Number of committed KV positions (tokens forwarded so far), or -1 for NULL. */
+int32_t kie_position(const kie_ctx* ctx);
+
+/* The pending token (fed to the next forward), or -1 if none / NULL ctx. */
+int32_t kie_pending(const kie_ctx* ctx);
+
+/* Fill *info for a context whose weights are loaded. Errors: INVALID_ARG, STATE. */
+kie_status kie_get_info(const kie_ctx* ctx, kie_info* info);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KIE_H_ */

@@ -1,0 +1,901 @@
+// Host side of libkie: context, weight packer, launcher and the C ABI.
+//
+// The packer lays every matrix out as the per-CTA "weight tape" that the
+// persistent kernel streams with TMA bulk copies (tile format in
+// kie_internal.h); the launcher runs a whole prefill or n-token decode as ONE
+// cooperative launch, so the host is crossed once per call instead of once per
+// kernel (the pages put a kernel launch at ~4.5 us and count >1,100 us of
+// launch overhead per token for an unfused 25-layer stack: "メモリの壁を打破する：
+// 標準的なGPUで3,000 tokens/sの推論を実現する", section "マイクロ秒が失われる場所").
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "../../include/kie.h"
+#include "kie_internal.h"
+
+namespace kie {
+int kernel_smem_bytes(int vec_floats, int n_stages);
+int kernel_max_stages();
+const void* kernel_entry();
+}  // namespace kie
+
+using namespace kie;
+
+namespace {
+
+thread_local std::string g_create_error;
+
+}  // namespace
+
+struct kie_ctx {
+  kie_config cfg{};
+  int device = 0;
+  int sms = 0;
+  int grid = 0;
+  int n_stages = 0;
+  int vec_floats = 0;
+  int smem = 0;
+  int max_chunks = 0;
+  int hbuf = 0;
+  int slots = 0;
+  SegShape shp[SK_COUNT]{};
+  // device memory
+  std::vector<void*> allocs;
+  unsigned char* tape = nullptr;
+  size_t tape_bytes = 0;
+  SegDesc* desc = nullptr;
+  __half *embed = nullptr, *attn_norm = nullptr, *mlp_norm = nullptr, *final_norm = nullptr,
+         *router = nullptr;
+  __half *kcache = nullptr, *vcache = nullptr;
+  float2* rope = nullptr;
+  float *x = nullptr, *qkv = nullptr, *o = nullptr, *h = nullptr, *apart = nullptr;
+  unsigned char* syncblk = nullptr;  // Ctrl + acnt[hk], cleared before every launch
+  size_t syncblk_bytes = 0;
+  Cand* cand = nullptr;
+  int *tok_dev = nullptr, *forced_dev = nullptr;
+  float* margins_dev = nullptr;
+  // state
+  bool loaded = false;
+  bool poisoned = false;
+  int32_t pos = 0;
+  int32_t pending = -1;
+  int64_t launches = 0;
+  int64_t stream_bytes = 0;
+  std::string err;
+};
+
+namespace {
+
+kie_status fail(kie_ctx* c, kie_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  if (c) c->err = buf;
+  else g_create_error = buf;
+  return s;
+}
+
+#define CUDA_TRY(ctx, call)                                                                  \
+  do {                                                                                       \
+    cudaError_t e_ = (call);                                                                 \
+    if (e_ != cudaSuccess) {                                                                 \
+      return fail((ctx), e_ == cudaErrorMemoryAllocation ? KIE_ERR_OOM : KIE_ERR_CUDA,      \
+                  "%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_), __FILE__, __LINE__); \
+    }                                                                                        \
+  } while (0)
+
+template <class T>
+kie_status dalloc(kie_ctx* c, T** p, size_t bytes) {
+  void* q = nullptr;
+  cudaError_t e = cudaMalloc(&q, bytes ? bytes : 16);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(c, e == cudaErrorMemoryAllocation ? KIE_ERR_OOM : KIE_ERR_CUDA,
+                "cudaMalloc(%zu) failed: %s", bytes, cudaGetErrorString(e));
+  }
+  c->allocs.push_back(q);
+  *p = static_cast<T*>(q);
+  return KIE_OK;
+}
+
+void dfree(kie_ctx* c, void* p) {
+  if (!p) return;
+  auto it = std::find(c->allocs.begin(), c->allocs.end(), p);
+  if (it != c->allocs.end()) c->allocs.erase(it);
+  cudaFree(p);
+}
+
+bool is_device_ptr(const void* p) {
+  cudaPointerAttributes a{};
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
+// Tile shape for a segment kind: rows per tile g and column chunks nk. Prefer
+// g >= 4 (the input vector chunk is reused across g rows) with the fewest
+// chunks; GU kinds need an even g so (gate, up) pairs share a tile.
+SegShape choose_shape(int K, bool pairs) {
+  SegShape best{K, 0, 0, 0};
+  for (int nk = 1; nk <= 64; ++nk) {
+    if (K % nk) continue;
+    const int kc = K / nk;
+    if (kc % 8) continue;
+    int g = std::min(kMaxRowsPerTile, kStageBytes / (2 * kc));
+    if (pairs) g &= ~1;
+    if (g < 1) continue;
+    if (g >= 4) return SegShape{K, g, nk, kc};
+    if (g > best.g) best = SegShape{K, g, nk, kc};
+  }
+  return best;
+}
+
+int seg_rows_per_unit(int kind) { return (kind == SK_GU || kind == SK_SGU || kind == SK_EGU) ? 2 : 1; }
+
+struct Tensor {
+  const void* data;
+  int64_t rows, cols;
+  bool on_dev;
+};
+
+}  // namespace
+
+// ------------------------------------------------------------------- packing
+
+__global__ void pack_rows_kernel(const unsigned long long* __restrict__ src,
+                                 const unsigned long long* __restrict__ dst, const int* __restrict__ n16,
+                                 long long count) {
+  const int lane = threadIdx.x & 31;
+  long long w = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const long long stride = (long long)gridDim.x * (blockDim.x / 32);
+  for (; w < count; w += stride) {
+    const uint4* s = reinterpret_cast<const uint4*>(src[w]);
+    uint4* d = reinterpret_cast<uint4*>(dst[w]);
+    const int n = n16[w];
+    for (int i = lane; i < n; i += 32) d[i] = s[i];
+  }
+}
+
+namespace {
+
+struct Planner {
+  kie_ctx* c;
+  const kie_config& k;
+  int G;
+  int slots;
+  std::vector<SegDesc> desc;  // [G][L*slots + 1]
+  std::vector<size_t> cta_bytes;
+
+  Planner(kie_ctx* ctx) : c(ctx), k(ctx->cfg), G(ctx->grid), slots(ctx->slots) {
+    desc.assign((size_t)G * (k.n_layers * slots + 1), SegDesc{0, 0, 0});
+    cta_bytes.assign(G, 0);
+  }
+
+  // rows of kind over the (virtual) row space, split into G near-equal ranges;
+  // the CTAs that get one extra unit rotate with `rot` so no CTA is always heavy.
+  void assign(int l, int slot, int kind, int rows, int rot) {
+    const int per = seg_rows_per_unit(kind);
+    const int U = rows / per;
+    const int b = U / G, rem = U % G;
+    for (int ci = 0; ci < G; ++ci) {
+      const int rank = (ci + rot) % G;
+      const int u0 = rank * b + std::min(rank, rem);
+      const int nu = b + (rank < rem ? 1 : 0);
+      SegDesc& d = desc[(size_t)ci * (k.n_layers * slots + 1) + (size_t)l * slots + slot];
+      d.row0 = u0 * per;
+      d.nrows = nu * per;
+    }
+    (void)kind;
+  }
+};
+
+}  // namespace
+
+extern "C" {
+
+kie_status kie_create(const kie_config* cfg, int device, kie_ctx** out) {
+  g_create_error.clear();
+  if (!cfg || !out) return fail(nullptr, KIE_ERR_INVALID_ARG, "null argument");
+  *out = nullptr;
+  const kie_config& k = *cfg;
+  const bool moe = k.n_experts > 0;
+  if (k.n_layers < 1 || k.d_model < 8 || k.n_heads < 1 || k.n_kv_heads < 1 || k.head_dim < 2 ||
+      k.vocab < 2 || k.max_ctx < 1)
+    return fail(nullptr, KIE_ERR_INVALID_ARG, "non-positive model dimension");
+  if (k.d_model % 8 || (k.n_heads * k.head_dim) % 8)
+    return fail(nullptr, KIE_ERR_INVALID_ARG, "d_model and n_heads*head_dim must be multiples of 8");
+  if (!(k.head_dim == 64 || k.head_dim == 128))
+    return fail(nullptr, KIE_ERR_INVALID_ARG, "head_dim must be 64 or 128");
+  if (k.n_kv_heads > k.n_heads)
+    return fail(nullptr, KIE_ERR_INVALID_ARG, "n_kv_heads > n_heads");
+  for (int g = 0; g < k.n_kv_heads; ++g) {
+    const int lo = (g * k.n_heads + k.n_kv_heads - 1) / k.n_kv_heads;
+    const int hi = ((g + 1) * k.n_heads + k.n_kv_heads - 1) / k.n_kv_heads;
+    if (hi - lo > kMaxHeadsPerGroup || hi - lo < 1)
+      return fail(nullptr, KIE_ERR_INVALID_ARG, "KV head %d serves %d query heads (1..%d allowed)", g,
+                  hi - lo, kMaxHeadsPerGroup);
+  }
+  if (moe) {
+    if (k.ffn != 0 || k.top_k < 1 || k.top_k > kMaxTopK || k.top_k > k.n_experts ||
+        k.n_experts > kMaxExperts || k.ffn_expert < 8 || k.ffn_shared < 8 || k.ffn_expert % 8 ||
+        k.ffn_shared % 8)
+      return fail(nullptr, KIE_ERR_INVALID_ARG, "bad MoE shape");
+  } else {
+    if (k.ffn < 8 || k.ffn % 8 || k.top_k || k.ffn_expert || k.ffn_shared)
+      return fail(nullptr, KIE_ERR_INVALID_ARG, "bad dense FFN shape");
+  }
+  if (!(k.rms_eps >= 0.f) || !(k.rope_theta > 0.f))
+    return fail(nullptr, KIE_ERR_INVALID_ARG, "bad rms_eps / rope_theta");
+
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+    cudaGetLastError();
+    return fail(nullptr, KIE_ERR_INVALID_ARG, "no CUDA device %d", device);
+  }
+  kie_ctx* c = new (std::nothrow) kie_ctx();
+  if (!c) return fail(nullptr, KIE_ERR_OOM, "host allocation failed");
+  c->cfg = k;
+  c->device = device;
+  auto bail = [&](kie_status s) {
+    g_create_error = c->err;
+    kie_destroy(c);
+    return s;
+  };
+  if (cudaSetDevice(device) != cudaSuccess) return bail(fail(c, KIE_ERR_CUDA, "cudaSetDevice failed"));
+  cudaDeviceProp prop{};
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess)
+    return bail(fail(c, KIE_ERR_CUDA, "cudaGetDeviceProperties failed"));
+  if (prop.major < 10) return bail(fail(c, KIE_ERR_CUDA, "device %s is not sm_100", prop.name));
+  if (!prop.cooperativeLaunch) return bail(fail(c, KIE_ERR_CUDA, "no cooperative launch support"));
+  c->sms = prop.multiProcessorCount;
+
+  const int hq = k.n_heads, hk = k.n_kv_heads, dh = k.head_dim, d = k.d_model;
+  c->hbuf = moe ? (k.ffn_shared + k.top_k * k.ffn_expert) : k.ffn;
+  int vf = std::max({d, hq * dh, c->hbuf, kConsumerWarps * kMaxHeadsPerGroup * dh});
+  vf = (vf + 3) & ~3;
+  c->vec_floats = vf;
+  const int fixed = kernel_smem_bytes(vf, 0);
+  const int optin = (int)prop.sharedMemPerBlockOptin;
+  int ns = (optin - fixed) / kStageBytes;
+  ns = std::min(ns, kernel_max_stages());
+  if (ns < 3) return bail(fail(c, KIE_ERR_INVALID_ARG, "shape needs too much shared memory"));
+  c->n_stages = ns;
+  c->smem = kernel_smem_bytes(vf, ns);
+  if (cudaFuncSetAttribute(kernel_entry(), cudaFuncAttributeMaxDynamicSharedMemorySize, c->smem) !=
+      cudaSuccess)
+    return bail(fail(c, KIE_ERR_CUDA, "cudaFuncSetAttribute(smem=%d) failed: %s", c->smem,
+                     cudaGetErrorString(cudaGetLastError())));
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel_entry(), kThreads, c->smem) !=
+          cudaSuccess ||
+      per_sm < 1)
+    return bail(fail(c, KIE_ERR_CUDA, "kernel does not fit on an SM (smem %d)", c->smem));
+  c->grid = c->sms;  // one CTA per SM; the ring takes the SM's shared memory
+  c->slots = slots_per_layer(moe ? k.n_experts : 0);
+
+  const int nwarps = c->grid * kConsumerWarps;
+  c->max_chunks = std::min((k.max_ctx + kAttnSub - 1) / kAttnSub, nwarps / hk + 2);
+
+  kie_status s;
+  const size_t kv = (size_t)k.n_layers * hk * k.max_ctx * dh * sizeof(__half);
+  if ((s = dalloc(c, &c->kcache, kv)) || (s = dalloc(c, &c->vcache, kv))) return bail(s);
+  if ((s = dalloc(c, &c->rope, (size_t)k.max_ctx * (dh / 2) * sizeof(float2)))) return bail(s);
+  {
+    std::vector<float2> tab((size_t)k.max_ctx * (dh / 2));
+    for (int p = 0; p < k.max_ctx; ++p)
+      for (int i = 0; i < dh / 2; ++i) {
+        const double phi = (double)p * std::pow((double)k.rope_theta, -2.0 * i / dh);
+        tab[(size_t)p * (dh / 2) + i] = make_float2((float)std::cos(phi), (float)std::sin(phi));
+      }
+    if (cudaMemcpy(c->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice) !=
+        cudaSuccess)
+      return bail(fail(c, KIE_ERR_CUDA, "rope table upload failed"));
+  }
+  if ((s = dalloc(c, &c->x, (size_t)d * 4)) ||
+      (s = dalloc(c, &c->qkv, (size_t)(hq + 2 * hk) * dh * 4)) ||
+      (s = dalloc(c, &c->o, (size_t)hq * dh * 4)) || (s = dalloc(c, &c->h, (size_t)c->hbuf * 4)) ||
+      (s = dalloc(c, &c->apart, (size_t)hq * c->max_chunks * (dh + 4) * 4)) ||
+      (s = dalloc(c, &c->cand, (size_t)c->grid * sizeof(Cand))) ||
+      (s = dalloc(c, &c->tok_dev, (size_t)k.max_ctx * 4)) ||
+      (s = dalloc(c, &c->forced_dev, (size_t)k.max_ctx * 4)) ||
+      (s = dalloc(c, &c->margins_dev, (size_t)k.max_ctx * 4)))
+    return bail(s);
+  c->syncblk_bytes = sizeof(Ctrl) + (size_t)hk * sizeof(unsigned);
+  if ((s = dalloc(c, &c->syncblk, c->syncblk_bytes))) return bail(s);
+  if (cudaMemset(c->syncblk, 0, c->syncblk_bytes) != cudaSuccess)
+    return bail(fail(c, KIE_ERR_CUDA, "memset failed"));
+  *out = c;
+  return KIE_OK;
+}
+
+kie_status kie_destroy(kie_ctx* c) {
+  if (!c) return KIE_OK;
+  cudaSetDevice(c->device);
+  for (void* p : c->allocs) cudaFree(p);
+  c->allocs.clear();
+  delete c;
+  return KIE_OK;
+}
+
+const char* kie_last_error(const kie_ctx* c) {
+  if (!c) return g_create_error.c_str();
+  return c->err.c_str();
+}
+
+int32_t kie_position(const kie_ctx* c) { return c ? c->pos : -1; }
+int32_t kie_pending(const kie_ctx* c) { return c ? c->pending : -1; }
+
+kie_status kie_reset(kie_ctx* c) {
+  if (!c) return KIE_ERR_INVALID_ARG;
+  c->err.clear();
+  cudaSetDevice(c->device);
+  cudaError_t e = cudaMemset(c->syncblk, 0, c->syncblk_bytes);
+  if (e != cudaSuccess) return fail(c, KIE_ERR_CUDA, "reset memset failed: %s", cudaGetErrorString(e));
+  c->pos = 0;
+  c->pending = -1;
+  c->poisoned = false;
+  return KIE_OK;
+}
+
+kie_status kie_rewind(kie_ctx* c, int32_t pos, int32_t pending) {
+  if (!c) return KIE_ERR_INVALID_ARG;
+  c->err.clear();
+  if (c->poisoned) return fail(c, KIE_ERR_STATE, "context is poisoned; call kie_reset");
+  if (!c->loaded) return fail(c, KIE_ERR_STATE, "weights not loaded");
+  if (pos < 0 || pos > c->pos) return fail(c, KIE_ERR_INVALID_ARG, "rewind to %d outside [0, %d]", pos, c->pos);
+  if (pending < 0 || pending >= c->cfg.vocab)
+    return fail(c, KIE_ERR_INVALID_ARG, "pending token %d outside [0, %d)", pending, c->cfg.vocab);
+  c->pos = pos;
+  c->pending = pending;
+  return KIE_OK;
+}
+
+kie_status kie_get_info(const kie_ctx* c, kie_info* info) {
+  if (!c || !info) return KIE_ERR_INVALID_ARG;
+  if (!c->loaded) return KIE_ERR_STATE;
+  const kie_config& k = c->cfg;
+  info->grid = c->grid;
+  info->threads = kThreads;
+  info->n_stages = c->n_stages;
+  info->stage_bytes = kStageBytes;
+  info->smem_bytes = c->smem;
+  info->barriers_per_token = 5 * k.n_layers + 1;
+  info->stream_bytes = c->stream_bytes;
+  info->kv_bytes_per_pos = 2LL * k.n_layers * k.n_kv_heads * k.head_dim * 2;
+  info->resident_bytes = (int64_t)c->tape_bytes;
+  info->launches = c->launches;
+  return KIE_OK;
+}
+
+kie_status kie_load_weights(kie_ctx* c, const kie_tensor* tensors, int n, void* stream) {
+  if (!c) return KIE_ERR_INVALID_ARG;
+  c->err.clear();
+  if (!tensors || n <= 0) return fail(c, KIE_ERR_INVALID_ARG, "no tensors");
+  cudaSetDevice(c->device);
+  cudaStream_t st = (cudaStream_t)stream;
+  const kie_config& k = c->cfg;
+  const bool moe = k.n_experts > 0;
+  const int d = k.d_model, hq = k.n_heads, hk = k.n_kv_heads, dh = k.head_dim, L = k.n_layers;
+
+  // expected tensors
+  std::map<std::string, std::pair<int64_t, int64_t>> want;
+  auto W = [&](const std::string& nm, int64_t r, int64_t cc) { want[nm] = {r, cc}; };
+  W("embed", k.vocab, d);
+  W("lm_head", k.vocab, d);
+  W("final_norm", d, 1);
+  for (int l = 0; l < L; ++l) {
+    const std::string p = "layers." + std::to_string(l) + ".";
+    W(p + "attn_norm", d, 1);
+    W(p + "mlp_norm", d, 1);
+    W(p + "wq", (int64_t)hq * dh, d);
+    W(p + "wk", (int64_t)hk * dh, d);
+    W(p + "wv", (int64_t)hk * dh, d);
+    W(p + "wo", d, (int64_t)hq * dh);
+    if (!moe) {
+      W(p + "w_gate", k.ffn, d);
+      W(p + "w_up", k.ffn, d);
+      W(p + "w_down", d, k.ffn);
+    } else {
+      W(p + "router", k.n_experts, d);
+      for (int e = 0; e < k.n_experts; ++e) {
+        const std::string q = p + "experts." + std::to_string(e) + ".";
+        W(q + "w_gate", k.ffn_expert, d);
+        W(q + "w_up", k.ffn_expert, d);
+        W(q + "w_down", d, k.ffn_expert);
+      }
+      W(p + "shared.w_gate", k.ffn_shared, d);
+      W(p + "shared.w_up", k.ffn_shared, d);
+      W(p + "shared.w_down", d, k.ffn_shared);
+    }
+  }
+  std::map<std::string, Tensor> got;
+  for (int i = 0; i < n; ++i) {
+    const kie_tensor& t = tensors[i];
+    if (!t.name || !t.data) return fail(c, KIE_ERR_INVALID_ARG, "tensor %d has a null name or data", i);
+    auto it = want.find(t.name);
+    if (it == want.end()) return fail(c, KIE_ERR_INVALID_ARG, "unexpected tensor '%s'", t.name);
+    if (got.count(t.name)) return fail(c, KIE_ERR_INVALID_ARG, "tensor '%s' given twice", t.name);
+    int64_t r = t.shape[0], cc = t.shape[1];
+    const bool vec = it->second.second == 1;
+    if (vec && r == 1 && cc == it->second.first) std::swap(r, cc);
+    if (r != it->second.first || cc != it->second.second)
+      return fail(c, KIE_ERR_INVALID_ARG, "tensor '%s' has shape [%lld, %lld], expected [%lld, %lld]",
+                  t.name, (long long)t.shape[0], (long long)t.shape[1], (long long)it->second.first,
+                  (long long)it->second.second);
+    if (t.on_device && !is_device_ptr(t.data))
+      return fail(c, KIE_ERR_INVALID_ARG, "tensor '%s' marked on_device but is not device memory", t.name);
+    if (t.on_device && (reinterpret_cast<uintptr_t>(t.data) & 15))
+      return fail(c, KIE_ERR_INVALID_ARG, "device tensor '%s' is not 16-byte aligned", t.name);
+    got[t.name] = Tensor{t.data, r, cc, t.on_device != 0};
+  }
+  for (auto& kv : want)
+    if (!got.count(kv.first)) return fail(c, KIE_ERR_INVALID_ARG, "missing tensor '%s'", kv.first.c_str());
+
+  // release a previous load
+  dfree(c, c->tape); c->tape = nullptr;
+  dfree(c, c->desc); c->desc = nullptr;
+  dfree(c, c->embed); c->embed = nullptr;
+  dfree(c, c->attn_norm); c->attn_norm = nullptr;
+  dfree(c, c->mlp_norm); c->mlp_norm = nullptr;
+  dfree(c, c->final_norm); c->final_norm = nullptr;
+  dfree(c, c->router); c->router = nullptr;
+  c->loaded = false;
+
+  // stage host tensors on the device (device tensors are read in place)
+  size_t stage_bytes = 0;
+  std::map<std::string, size_t> soff;
+  for (auto& kv : got)
+    if (!kv.second.on_dev) {
+      soff[kv.first] = stage_bytes;
+      stage_bytes += ((size_t)kv.second.rows * kv.second.cols * 2 + 255) & ~(size_t)255;
+    }
+  unsigned char* staging = nullptr;
+  kie_status s;
+  if (stage_bytes && (s = dalloc(c, &staging, stage_bytes))) return s;
+  std::map<std::string, const unsigned char*> dptr;
+  for (auto& kv : got) {
+    if (kv.second.on_dev) {
+      dptr[kv.first] = static_cast<const unsigned char*>(kv.second.data);
+    } else {
+      unsigned char* dst = staging + soff[kv.first];
+      const size_t bytes = (size_t)kv.second.rows * kv.second.cols * 2;
+      cudaError_t e = cudaMemcpyAsync(dst, kv.second.data, bytes, cudaMemcpyHostToDevice, st);
+      if (e != cudaSuccess) {
+        dfree(c, staging);
+        return fail(c, KIE_ERR_CUDA, "upload of '%s' failed: %s", kv.first.c_str(), cudaGetErrorString(e));
+      }
+      dptr[kv.first] = dst;
+    }
+  }
+
+  // segment shapes
+  const int ffs = k.ffn_shared, ffe = k.ffn_expert;
+  c->shp[SK_QKV] = choose_shape(d, false);
+  c->shp[SK_O] = choose_shape(hq * dh, false);
+  c->shp[SK_LM] = choose_shape(d, false);
+  if (!moe) {
+    c->shp[SK_GU] = choose_shape(d, true);
+    c->shp[SK_DOWN] = choose_shape(k.ffn, false);
+  } else {
+    c->shp[SK_SGU] = choose_shape(d, true);
+    c->shp[SK_EGU] = choose_shape(d, true);
+    c->shp[SK_SDOWN] = choose_shape(ffs, false);
+    c->shp[SK_EDOWN] = choose_shape(ffe, false);
+  }
+
+  // row assignment
+  Planner pl(c);
+  const int G = c->grid;
+  for (int l = 0; l < L; ++l) {
+    const int rot = (int)(((long long)l * 53) % G);
+    pl.assign(l, 0, SK_QKV, (hq + 2 * hk) * dh, rot);
+    pl.assign(l, 1, SK_O, d, (rot + 17) % G);
+    if (!moe) {
+      pl.assign(l, 2, SK_GU, 2 * k.ffn, (rot + 31) % G);
+      pl.assign(l, 3, SK_DOWN, d, (rot + 71) % G);
+    } else {
+      pl.assign(l, 2, SK_SGU, 2 * ffs, (rot + 31) % G);
+      pl.assign(l, 3, SK_SDOWN, d, (rot + 71) % G);
+      for (int e = 0; e < k.n_experts; ++e) {
+        pl.assign(l, 4 + e, SK_EGU, 2 * ffe, (rot + 97 + 7 * e) % G);
+        pl.assign(l, 4 + k.n_experts + e, SK_EDOWN, d, (rot + 71) % G);  // same rows as SDOWN
+      }
+    }
+  }
+  pl.assign(L, 0, SK_LM, k.vocab, 0);
+
+  auto kind_of = [&](int l, int slot) -> int {
+    if (l == L) return SK_LM;
+    if (slot == 0) return SK_QKV;
+    if (slot == 1) return SK_O;
+    if (!moe) return slot == 2 ? SK_GU : SK_DOWN;
+    if (slot == 2) return SK_SGU;
+    if (slot == 3) return SK_SDOWN;
+    return slot < 4 + k.n_experts ? SK_EGU : SK_EDOWN;
+  };
+  const int per_cta = L * c->slots + 1;
+  // partial-slot capacity per phase
+  {
+    int worst = 0;
+    for (int ci = 0; ci < G; ++ci) {
+      const SegDesc* D = &pl.desc[(size_t)ci * per_cta];
+      for (int l = 0; l < L; ++l) {
+        const SegDesc* Dl = D + (size_t)l * c->slots;
+        worst = std::max(worst, Dl[0].nrows * c->shp[SK_QKV].nk);
+        worst = std::max(worst, Dl[1].nrows * c->shp[SK_O].nk);
+        if (!moe) {
+          worst = std::max(worst, Dl[2].nrows * c->shp[SK_GU].nk);
+          worst = std::max(worst, Dl[3].nrows * c->shp[SK_DOWN].nk);
+        } else {
+          int eg = 0, ed = 0;
+          for (int e = 0; e < k.n_experts; ++e) {
+            eg = std::max(eg, Dl[4 + e].nrows);
+            ed = std::max(ed, Dl[4 + k.n_experts + e].nrows);
+          }
+          worst = std::max(worst, Dl[2].nrows * c->shp[SK_SGU].nk + k.top_k * eg * c->shp[SK_EGU].nk);
+          worst = std::max(worst, Dl[3].nrows * (c->shp[SK_SDOWN].nk + k.top_k * c->shp[SK_EDOWN].nk));
+        }
+      }
+      worst = std::max(worst, D[(size_t)L * c->slots].nrows * c->shp[SK_LM].nk);
+    }
+    if (worst > kPartFloats) {
+      dfree(c, staging);
+      return fail(c, KIE_ERR_INVALID_ARG, "a CTA would hold %d partial sums (max %d)", worst, kPartFloats);
+    }
+  }
+
+  // tape offsets: each CTA's region contiguous, segments in execution order
+  size_t off = 0;
+  for (int ci = 0; ci < G; ++ci) {
+    for (int l = 0; l <= L; ++l) {
+      const int ns = (l == L) ? 1 : c->slots;
+      for (int slot = 0; slot < ns; ++slot) {
+        SegDesc& sd = pl.desc[(size_t)ci * per_cta + (size_t)l * c->slots + slot];
+        sd.off = off;
+        off += (size_t)sd.nrows * c->shp[kind_of(l, slot)].K * 2;
+      }
+    }
+  }
+  c->tape_bytes = off;
+  if ((s = dalloc(c, &c->tape, off))) {
+    dfree(c, staging);
+    return s;
+  }
+
+  // row-copy list: virtual row -> source row pointer
+  auto rowptr = [&](int l, int slot, int row) -> const unsigned char* {
+    const int kind = kind_of(l, slot);
+    const std::string p = "layers." + std::to_string(l) + ".";
+    switch (kind) {
+      case SK_QKV:
+        if (row < hq * dh) return dptr[p + "wq"] + (size_t)row * d * 2;
+        if (row < (hq + hk) * dh) return dptr[p + "wk"] + (size_t)(row - hq * dh) * d * 2;
+        return dptr[p + "wv"] + (size_t)(row - (hq + hk) * dh) * d * 2;
+      case SK_O: return dptr[p + "wo"] + (size_t)row * hq * dh * 2;
+      case SK_GU: return dptr[p + ((row & 1) ? "w_up" : "w_gate")] + (size_t)(row / 2) * d * 2;
+      case SK_DOWN: return dptr[p + "w_down"] + (size_t)row * k.ffn * 2;
+      case SK_SGU: return dptr[p + ((row & 1) ? "shared.w_up" : "shared.w_gate")] + (size_t)(row / 2) * d * 2;
+      case SK_SDOWN: return dptr[p + "shared.w_down"] + (size_t)row * ffs * 2;
+      case SK_EGU: {
+        const int e = slot - 4;
+        const std::string q = p + "experts." + std::to_string(e) + ".";
+        return dptr[q + ((row & 1) ? "w_up" : "w_gate")] + (size_t)(row / 2) * d * 2;
+      }
+      case SK_EDOWN: {
+        const int e = slot - 4 - k.n_experts;
+        return dptr[p + "experts." + std::to_string(e) + ".w_down"] + (size_t)row * ffe * 2;
+      }
+      default: return dptr["lm_head"] + (size_t)row * d * 2;
+    }
+  };
+  // cache the string lookups per (layer, slot) by resolving row 0 and 1 bases lazily:
+  // the list is built layer by layer to bound host memory.
+  std::vector<unsigned long long> hsrc, hdst;
+  std::vector<int> hn;
+  unsigned long long* dsrc = nullptr;
+  unsigned long long* ddst = nullptr;
+  int* dn = nullptr;
+  size_t cap = 0;
+  auto flush = [&]() -> kie_status {
+    const size_t m = hsrc.size();
+    if (!m) return KIE_OK;
+    if (m > cap) {
+      dfree(c, dsrc); dfree(c, ddst); dfree(c, dn);
+      dsrc = ddst = nullptr; dn = nullptr;
+      cap = m;
+      kie_status s2;
+      if ((s2 = dalloc(c, &dsrc, m * 8)) || (s2 = dalloc(c, &ddst, m * 8)) || (s2 = dalloc(c, &dn, m * 4)))
+        return s2;
+    }
+    CUDA_TRY(c, cudaMemcpyAsync(dsrc, hsrc.data(), m * 8, cudaMemcpyHostToDevice, st));
+    CUDA_TRY(c, cudaMemcpyAsync(ddst, hdst.data(), m * 8, cudaMemcpyHostToDevice, st));
+    CUDA_TRY(c, cudaMemcpyAsync(dn, hn.data(), m * 4, cudaMemcpyHostToDevice, st));
+    const int blocks = (int)std::min<size_t>((m + 7) / 8, 4096);
+    pack_rows_kernel<<<blocks, 256, 0, st>>>(dsrc, ddst, dn, (long long)m);
+    CUDA_TRY(c, cudaGetLastError());
+    c->launches++;
+    CUDA_TRY(c, cudaStreamSynchronize(st));  // host vectors are reused
+    hsrc.clear(); hdst.clear(); hn.clear();
+    return KIE_OK;
+  };
+  kie_status ps = KIE_OK;
+  for (int l = 0; l <= L && ps == KIE_OK; ++l) {
+    const int nsl = (l == L) ? 1 : c->slots;
+    for (int slot = 0; slot < nsl; ++slot) {
+      const SegShape& sh = c->shp[kind_of(l, slot)];
+      // resolve two base pointers per slot once (even/odd rows for GU kinds)
+      for (int ci = 0; ci < G; ++ci) {
+        const SegDesc& sd = pl.desc[(size_t)ci * per_cta + (size_t)l * c->slots + slot];
+        const int ngroups = (sd.nrows + sh.g - 1) / sh.g;
+        for (int gi = 0; gi < ngroups; ++gi) {
+          const int gp = std::min(sh.g, sd.nrows - gi * sh.g);
+          for (int kj = 0; kj < sh.nk; ++kj) {
+            for (int r = 0; r < gp; ++r) {
+              const int row = sd.row0 + gi * sh.g + r;
+              const unsigned char* src = rowptr(l, slot, row) + (size_t)kj * sh.kc * 2;
+              unsigned char* dst = c->tape + sd.off + (size_t)gi * sh.g * sh.K * 2 +
+                                   (size_t)kj * gp * sh.kc * 2 + (size_t)r * sh.kc * 2;
+              hsrc.push_back((unsigned long long)src);
+              hdst.push_back((unsigned long long)dst);
+              hn.push_back(sh.kc / 8);
+            }
+          }
+        }
+      }
+    }
+    ps = flush();
+  }
+  if (ps != KIE_OK) {
+    dfree(c, staging);
+    return ps;
+  }
+  dfree(c, dsrc); dfree(c, ddst); dfree(c, dn);
+
+  // descriptors and the small tensors kept outside the tape
+  if ((s = dalloc(c, &c->desc, pl.desc.size() * sizeof(SegDesc)))) return s;
+  CUDA_TRY(c, cudaMemcpyAsync(c->desc, pl.desc.data(), pl.desc.size() * sizeof(SegDesc),
+                              cudaMemcpyHostToDevice, st));
+  if ((s = dalloc(c, &c->embed, (size_t)k.vocab * d * 2)) ||
+      (s = dalloc(c, &c->attn_norm, (size_t)L * d * 2)) || (s = dalloc(c, &c->mlp_norm, (size_t)L * d * 2)) ||
+      (s = dalloc(c, &c->final_norm, (size_t)d * 2)))
+    return s;
+  CUDA_TRY(c, cudaMemcpyAsync(c->embed, dptr["embed"], (size_t)k.vocab * d * 2, cudaMemcpyDeviceToDevice, st));
+  CUDA_TRY(c, cudaMemcpyAsync(c->final_norm, dptr["final_norm"], (size_t)d * 2, cudaMemcpyDeviceToDevice, st));
+  for (int l = 0; l < L; ++l) {
+    const std::string p = "layers." + std::to_string(l) + ".";
+    CUDA_TRY(c, cudaMemcpyAsync(c->attn_norm + (size_t)l * d, dptr[p + "attn_norm"], (size_t)d * 2,
+                                cudaMemcpyDeviceToDevice, st));
+    CUDA_TRY(c, cudaMemcpyAsync(c->mlp_norm + (size_t)l * d, dptr[p + "mlp_norm"], (size_t)d * 2,
+                                cudaMemcpyDeviceToDevice, st));
+  }
+  if (moe) {
+    if ((s = dalloc(c, &c->router, (size_t)L * k.n_experts * d * 2))) return s;
+    for (int l = 0; l < L; ++l)
+      CUDA_TRY(c, cudaMemcpyAsync(c->router + (size_t)l * k.n_experts * d,
+                                  dptr["layers." + std::to_string(l) + ".router"],
+                                  (size_t)k.n_experts * d * 2, cudaMemcpyDeviceToDevice, st));
+  }
+  CUDA_TRY(c, cudaStreamSynchronize(st));
+  dfree(c, staging);
+
+  // algorithmic weight bytes streamed per decoded token
+  int64_t sb = 0;
+  const int64_t qkvb = (int64_t)(hq + 2 * hk) * dh * d * 2, ob = (int64_t)d * hq * dh * 2;
+  if (!moe) {
+    sb = L * (qkvb + ob + 3LL * k.ffn * d * 2);
+  } else {
+    sb = L * (qkvb + ob + (int64_t)k.n_experts * d * 2 + 3LL * ffs * d * 2 + k.top_k * 3LL * ffe * d * 2);
+  }
+  sb += (int64_t)k.vocab * d * 2 + (2LL * L + 1) * d * 2 + (int64_t)d * 2;
+  c->stream_bytes = sb;
+  c->loaded = true;
+  c->pos = 0;
+  c->pending = -1;
+  c->poisoned = false;
+  return KIE_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+struct Run {
+  int first_token, n_steps, lm_from_step;
+  const int* forced;
+  int* out;
+  float* logits;
+  float* margins;
+  uint32_t timeout_ms;
+  int fault_cta, fault_barrier;
+  uint64_t* trace;
+  int trace_cap;
+};
+
+kie_status launch(kie_ctx* c, const Run& r, cudaStream_t st) {
+  const kie_config& k = c->cfg;
+  Params P{};
+  P.L = k.n_layers; P.d = k.d_model; P.hq = k.n_heads; P.hk = k.n_kv_heads; P.dh = k.head_dim;
+  P.ff = k.ffn; P.V = k.vocab; P.E = k.n_experts; P.top_k = k.top_k; P.ffe = k.ffn_expert;
+  P.ffs = k.ffn_shared; P.max_ctx = k.max_ctx; P.eps = k.rms_eps;
+  P.qkv_rows = (k.n_heads + 2 * k.n_kv_heads) * k.head_dim;
+  P.slots = c->slots;
+  P.tape = c->tape; P.desc = c->desc;
+  for (int i = 0; i < SK_COUNT; ++i) P.shp[i] = c->shp[i];
+  P.embed = c->embed; P.attn_norm = c->attn_norm; P.mlp_norm = c->mlp_norm;
+  P.final_norm = c->final_norm; P.router = c->router;
+  P.kcache = c->kcache; P.vcache = c->vcache; P.rope = c->rope;
+  P.x = c->x; P.qkv = c->qkv; P.o = c->o; P.h = c->h; P.apart = c->apart;
+  P.ctrl = reinterpret_cast<Ctrl*>(c->syncblk);
+  P.acnt = reinterpret_cast<unsigned*>(c->syncblk + sizeof(Ctrl));
+  P.cand = c->cand; P.max_chunks = c->max_chunks;
+  P.pos0 = c->pos; P.n_steps = r.n_steps; P.first_token = r.first_token; P.lm_from_step = r.lm_from_step;
+  P.forced = r.forced; P.out_tokens = r.out; P.logits_out = r.logits; P.margins_out = r.margins;
+  P.timeout_ns = (unsigned long long)(r.timeout_ms ? r.timeout_ms : 1000u) * 1000000ull;
+  P.fault_cta = r.fault_cta; P.fault_barrier = r.fault_barrier;
+  P.trace = reinterpret_cast<unsigned long long*>(r.trace); P.trace_cap = r.trace_cap;
+  P.n_stages = c->n_stages; P.vec_floats = c->vec_floats;
+
+  CUDA_TRY(c, cudaMemsetAsync(c->syncblk, 0, c->syncblk_bytes, st));
+  void* args[] = {&P};
+  cudaError_t e = cudaLaunchCooperativeKernel(kernel_entry(), dim3(c->grid), dim3(kThreads), args,
+                                              (size_t)c->smem, st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(c, KIE_ERR_CUDA, "cooperative launch failed: %s", cudaGetErrorString(e));
+  }
+  c->launches++;
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) {
+    c->poisoned = true;
+    return fail(c, KIE_ERR_CUDA, "decode kernel failed: %s", cudaGetErrorString(e));
+  }
+  Ctrl ctl{};
+  CUDA_TRY(c, cudaMemcpy(&ctl, c->syncblk, sizeof(Ctrl), cudaMemcpyDeviceToHost));
+  if (ctl.err) {
+    c->poisoned = true;
+    static const char* where[] = {"?", "grid barrier", "ring stage (full)", "ring stage (empty)",
+                                  "expert routing hand-off", "device check"};
+    const int w = (ctl.err_where >= 1 && ctl.err_where <= 5) ? ctl.err_where : 0;
+    return fail(c, (kie_status)ctl.err, "device %s at %s (cta %d, step %d); context poisoned",
+                ctl.err == KIE_ERR_TIMEOUT ? "timeout" : "check failed", where[w], ctl.err_cta,
+                ctl.err_step);
+  }
+  c->pending = ctl.final_token;
+  return KIE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kie_status kie_prefill(kie_ctx* c, const int32_t* tokens, int n, void* stream) {
+  if (!c) return KIE_ERR_INVALID_ARG;
+  c->err.clear();
+  if (c->poisoned) return fail(c, KIE_ERR_STATE, "context is poisoned; call kie_reset");
+  if (!c->loaded) return fail(c, KIE_ERR_STATE, "weights not loaded");
+  if (n < 0 || (n > 0 && !tokens)) return fail(c, KIE_ERR_INVALID_ARG, "bad token array");
+  if (n == 0) return KIE_OK;
+  if (is_device_ptr(tokens)) return fail(c, KIE_ERR_INVALID_ARG, "prefill tokens must be host memory");
+  for (int i = 0; i < n; ++i)
+    if (tokens[i] < 0 || tokens[i] >= c->cfg.vocab)
+      return fail(c, KIE_ERR_INVALID_ARG, "token %d at index %d outside [0, %d)", tokens[i], i, c->cfg.vocab);
+  std::vector<int32_t> seq;
+  if (c->pending >= 0) seq.push_back(c->pending);
+  for (int i = 0; i + 1 < n; ++i) seq.push_back(tokens[i]);
+  if ((int64_t)c->pos + (int64_t)seq.size() > c->cfg.max_ctx)
+    return fail(c, KIE_ERR_CONTEXT_FULL, "position %d + %zu tokens exceeds max_ctx %d", c->pos, seq.size(),
+                c->cfg.max_ctx);
+  cudaSetDevice(c->device);
+  cudaStream_t st = (cudaStream_t)stream;
+  const int kChunk = 8192;  // bounds the barrier counter of one launch
+  const int32_t new_pending = tokens[n - 1];
+  size_t i0 = 0;
+  const int32_t pos_before = c->pos, pend_before = c->pending;
+  while (i0 < seq.size()) {
+    const int m = (int)std::min<size_t>(kChunk, seq.size() - i0);
+    // forced[i] = token fed after step i
+    std::vector<int32_t> f(m);
+    for (int i = 0; i < m; ++i) f[i] = (i0 + i + 1 < seq.size()) ? seq[i0 + i + 1] : new_pending;
+    CUDA_TRY(c, cudaMemcpyAsync(c->forced_dev, f.data(), (size_t)m * 4, cudaMemcpyHostToDevice, st));
+    Run r{seq[i0], m, m, c->forced_dev, c->tok_dev, nullptr, nullptr, 0, -1, -1, nullptr, 0};
+    kie_status s = launch(c, r, st);
+    if (s != KIE_OK) {
+      if (!c->poisoned) { c->pos = pos_before; c->pending = pend_before; }
+      return s;
+    }
+    c->pos += m;
+    i0 += m;
+  }
+  c->pending = new_pending;
+  return KIE_OK;
+}
+
+kie_status kie_decode(kie_ctx* c, int n, int32_t* out_tokens, const kie_decode_opts* opts, void* stream) {
+  if (!c) return KIE_ERR_INVALID_ARG;
+  c->err.clear();
+  if (c->poisoned) return fail(c, KIE_ERR_STATE, "context is poisoned; call kie_reset");
+  if (!c->loaded) return fail(c, KIE_ERR_STATE, "weights not loaded");
+  if (n < 0) return fail(c, KIE_ERR_INVALID_ARG, "negative token count");
+  if (n == 0) return KIE_OK;
+  if (!out_tokens) return fail(c, KIE_ERR_INVALID_ARG, "out_tokens is null");
+  if (c->pending < 0) return fail(c, KIE_ERR_STATE, "no pending token: prefill first");
+  if ((int64_t)c->pos + n > c->cfg.max_ctx)
+    return fail(c, KIE_ERR_CONTEXT_FULL, "position %d + %d tokens exceeds max_ctx %d", c->pos, n, c->cfg.max_ctx);
+  kie_decode_opts o{};
+  o.fault_cta = -1;
+  o.fault_barrier = -1;
+  if (opts) o = *opts;
+  if (o.trace_out && o.trace_cap <= 0) return fail(c, KIE_ERR_INVALID_ARG, "trace_cap must be > 0");
+  cudaSetDevice(c->device);
+  cudaStream_t st = (cudaStream_t)stream;
+  const int V = c->cfg.vocab;
+
+  const int* forced = nullptr;
+  if (o.forced_tokens) {
+    std::vector<int32_t> f(n);
+    if (is_device_ptr(o.forced_tokens)) {
+      CUDA_TRY(c, cudaMemcpyAsync(f.data(), o.forced_tokens, (size_t)n * 4, cudaMemcpyDeviceToHost, st));
+      CUDA_TRY(c, cudaStreamSynchronize(st));
+    } else
+      std::memcpy(f.data(), o.forced_tokens, (size_t)n * 4);
+    for (int i = 0; i < n; ++i)
+      if (f[i] < -1 || f[i] >= V)
+        return fail(c, KIE_ERR_INVALID_ARG, "forced token %d at step %d outside [-1, %d)", f[i], i, V);
+    CUDA_TRY(c, cudaMemcpyAsync(c->forced_dev, f.data(), (size_t)n * 4, cudaMemcpyHostToDevice, st));
+    forced = c->forced_dev;
+  }
+  const bool out_dev = is_device_ptr(out_tokens);
+  float* logits = nullptr;
+  float* logits_tmp = nullptr;
+  if (o.logits_out) {
+    if (is_device_ptr(o.logits_out)) {
+      logits = o.logits_out;
+    } else {
+      kie_status s = dalloc(c, &logits_tmp, (size_t)n * V * 4);
+      if (s) return s;
+      logits = logits_tmp;
+    }
+  }
+  float* margins = nullptr;
+  if (o.margins_out) margins = is_device_ptr(o.margins_out) ? o.margins_out : c->margins_dev;
+  Run r{c->pending, n, 0, forced, out_dev ? out_tokens : c->tok_dev, logits, margins, o.timeout_ms,
+        o.fault_cta, o.fault_barrier, o.trace_out, o.trace_cap};
+  kie_status s = launch(c, r, st);
+  if (s == KIE_OK) {
+    if (!out_dev) {
+      cudaError_t e = cudaMemcpyAsync(out_tokens, c->tok_dev, (size_t)n * 4, cudaMemcpyDefault, st);
+      if (e == cudaSuccess && logits_tmp)
+        e = cudaMemcpyAsync(o.logits_out, logits_tmp, (size_t)n * V * 4, cudaMemcpyDefault, st);
+      if (e == cudaSuccess && o.margins_out && margins == c->margins_dev)
+        e = cudaMemcpyAsync(o.margins_out, margins, (size_t)n * 4, cudaMemcpyDefault, st);
+      if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+      if (e != cudaSuccess) s = fail(c, KIE_ERR_CUDA, "result copy failed: %s", cudaGetErrorString(e));
+    } else {
+      cudaError_t e = cudaSuccess;
+      if (logits_tmp) e = cudaMemcpyAsync(o.logits_out, logits_tmp, (size_t)n * V * 4, cudaMemcpyDefault, st);
+      if (e == cudaSuccess && o.margins_out && margins == c->margins_dev)
+        e = cudaMemcpyAsync(o.margins_out, margins, (size_t)n * 4, cudaMemcpyDefault, st);
+      if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+      if (e != cudaSuccess) s = fail(c, KIE_ERR_CUDA, "result copy failed: %s", cudaGetErrorString(e));
+    }
+    if (s == KIE_OK) c->pos += n;
+  }
+  if (logits_tmp) dfree(c, logits_tmp);
+  return s;
+}
+
+}  // extern "C"

@@ -1,0 +1,123 @@
+// Internal layout shared by the host side (packer, launcher) and the
+// persistent decode kernel. Not part of the public ABI (see include/kie.h).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace kie {
+
+// ---- launch geometry ------------------------------------------------------
+constexpr int kConsumerWarps = 8;                      // GEMV / attention warps
+constexpr int kConsumerThreads = kConsumerWarps * 32;  // named barrier 1 spans these
+constexpr int kThreads = kConsumerThreads + 32;        // + one producer (TMA) warp
+constexpr int kStageBytes = 16384;                     // one ring stage = one weight tile
+constexpr int kMaxRowsPerTile = 8;                     // rows of one tile (register-blocked)
+constexpr int kPartFloats = 2048;                      // per-CTA partial-sum slots per phase
+constexpr int kMaxHeadsPerGroup = 4;                   // query heads per KV head (GQA)
+constexpr int kMaxTopK = 4;                            // routed experts per token
+constexpr int kAttnSub = 32;                           // positions per attention sub-block
+constexpr int kMaxExperts = 64;
+
+// ---- weight tape ------------------------------------------------------------
+// The tape is one device buffer. CTA c owns a contiguous region holding, in
+// execution order, its slice of every weight matrix of one decode step. A
+// "segment" is one CTA's slice of one matrix: rows [row0, row0 + nrows) of the
+// matrix's (virtual) row space, stored as groups of `g` rows (the last group
+// may be shorter); each group is cut into `nk` column chunks of `kc` columns,
+// and each (group, chunk) tile is stored row-major [g'][kc] and is one TMA
+// bulk copy of g' * kc * 2 bytes.
+enum SegKind : int {
+  SK_QKV = 0,   // rows: [wq; wk; wv], K = d
+  SK_O = 1,     // rows: wo, K = hq*dh
+  SK_GU = 2,    // rows: gate_0, up_0, gate_1, up_1, ... (dense FFN), K = d
+  SK_DOWN = 3,  // rows: w_down, K = ffn
+  SK_SGU = 4,   // shared expert gate/up interleaved, K = d
+  SK_EGU = 5,   // routed expert gate/up interleaved, K = d
+  SK_SDOWN = 6, // shared expert down, K = ffs
+  SK_EDOWN = 7, // routed expert down, K = ffe
+  SK_LM = 8,    // lm_head, K = d
+  SK_COUNT = 9
+};
+
+struct SegShape {
+  int K;   // columns of the matrix (input length)
+  int g;   // rows per tile (full groups)
+  int nk;  // column chunks per group
+  int kc;  // columns per chunk (K / nk, multiple of 8)
+};
+
+struct SegDesc {
+  unsigned long long off;  // byte offset of this segment in the tape
+  int row0;                // first (virtual) row owned by this CTA
+  int nrows;               // rows owned (GU kinds: always even)
+};
+
+// Descriptor slots per layer: 0 QKV, 1 O, 2 GU|SGU, 3 DOWN|SDOWN,
+// 4..4+E-1 EGU[e], 4+E..4+2E-1 EDOWN[e]. The LM head is slot 0 of layer L.
+__host__ __device__ inline int slots_per_layer(int n_experts) { return 4 + 2 * n_experts; }
+
+// ---- device control block ---------------------------------------------------
+struct Ctrl {
+  unsigned int arrive;   // grid barrier arrivals (monotonic within one launch)
+  unsigned int abort;    // set to 1 by any CTA that gives up; all CTAs poll it
+  int err;               // first error code (kie_status value), 0 = none
+  int err_cta;           // CTA that recorded the error
+  int err_step;          // decode step
+  int err_where;         // 1 grid barrier, 2 ring full-wait, 3 ring empty-wait,
+                         // 4 route wait, 5 device check
+  int final_token;       // pending token after the last step
+  int pad;
+};
+
+struct Cand {  // per-CTA greedy candidate: best value, its index, second value
+  float v1;
+  int i1;
+  float v2;
+  int pad;
+};
+
+struct Params {
+  // model shape
+  int L, d, hq, hk, dh, ff, V, E, top_k, ffe, ffs, max_ctx;
+  float eps;
+  int qkv_rows;    // (hq + 2 hk) dh
+  int slots;       // descriptor slots per layer
+  // packed weights
+  const unsigned char* tape;
+  const SegDesc* desc;       // [grid][L * slots + 1]
+  SegShape shp[SK_COUNT];
+  const __half* embed;       // [V][d]
+  const __half* attn_norm;   // [L][d]
+  const __half* mlp_norm;    // [L][d]
+  const __half* final_norm;  // [d]
+  const __half* router;      // [L][E][d] (MoE) or null
+  // state
+  __half* kcache;            // [L][hk][max_ctx][dh]
+  __half* vcache;
+  const float2* rope;        // [max_ctx][dh/2] (cos, sin)
+  // scratch
+  float* x;                  // [d] residual stream
+  float* qkv;                // [qkv_rows] raw q|k|v
+  float* o;                  // [hq*dh] attention output
+  float* h;                  // [hbuf] FFN hidden (dense: ff; MoE: ffs + top_k*ffe)
+  float* apart;              // attention partials [hq][max_chunks][dh + 4]
+  unsigned int* acnt;        // [hk] per-KV-head arrival counters
+  Cand* cand;                // [grid]
+  Ctrl* ctrl;
+  int max_chunks;
+  // run
+  int pos0, n_steps, first_token, lm_from_step;
+  const int* forced;         // device [n_steps] or null
+  int* out_tokens;           // device [n_steps]
+  float* logits_out;         // device [n_steps][V] or null
+  float* margins_out;        // device [n_steps] or null
+  unsigned long long timeout_ns;
+  int fault_cta, fault_barrier;
+  unsigned long long* trace; // device [grid][trace_cap][2] or null
+  int trace_cap;
+  int n_stages;
+  int vec_floats;
+};
+
+}  // namespace kie
