@@ -28,7 +28,13 @@ math; the readings taken (all listed in the design notes) are:
 * Greedy: argmax with the lowest index on exact ties; the margin is the top
   value minus the second-largest value (0 on a tie).
 * No biases, no QK-norm, no logit scaling. Weights are fp16 and widened to
-  fp64 at use; K and V are kept unrounded in fp64.
+  fp64 at use.
+* The KV cache is fp16: the workload descriptions fix it ("KV cache fp16",
+  "prefilled into an fp16 KV cache") and the method attends "over an FP16 KV
+  cache". So K (after RoPE) and V are rounded to fp16 (round to nearest even)
+  when they enter the cache, in both the incremental and the full-sequence
+  form; every other step stays in fp64. ``kv_fp16=False`` keeps them
+  unrounded (for diagnosis).
 
 Everything is float64, single process; numpy's matrix product is used as the
 plain library primitive for y = W x (and X W^T in the full-sequence form).
@@ -180,17 +186,24 @@ def moe_ffn(xn, router, experts, shared, top_k: int) -> np.ndarray:
 
 # ---------------------------------------------------------------- the model
 
+def fp16_round(a) -> np.ndarray:
+    """Round to the nearest fp16 value (ties to even), returned as float64."""
+    return np.asarray(a, dtype=np.float64).astype(np.float16).astype(np.float64)
+
+
 class Decoder:
     """The whole decoder over fp16 weights from ``synthetic.make_weights``.
 
     ``cache_f64`` keeps a widened copy of each matrix after its first use
-    (memory for speed; the values are the same either way).
+    (memory for speed; the values are the same either way). ``kv_fp16``
+    rounds cached K and V to fp16 (the workloads' fp16 KV cache).
     """
 
-    def __init__(self, shape, weights: dict, cache_f64: bool = True):
+    def __init__(self, shape, weights: dict, cache_f64: bool = True, kv_fp16: bool = True):
         self.s = shape
         self.w16 = weights
         self._w64 = {} if cache_f64 else None
+        self.kv = fp16_round if kv_fp16 else f64
 
     def W(self, name: str) -> np.ndarray:
         if self._w64 is None:
@@ -245,6 +258,7 @@ class Decoder:
             k = (xn @ self.W(p + "wk").T).reshape(T, s.n_kv_heads, dh)
             v = (xn @ self.W(p + "wv").T).reshape(T, s.n_kv_heads, dh)
             q, k = rope(q, pos, s.rope_theta), rope(k, pos, s.rope_theta)
+            k, v = self.kv(k), self.kv(v)
             o = causal_attention(q, k, v).reshape(T, s.n_heads * dh)
             x = x + o @ self.W(p + "wo").T
             xn = rmsnorm(x, self.w16[p + "mlp_norm"], s.rms_eps)
@@ -275,8 +289,8 @@ class Decoder:
             k = (self.W(w + "wk") @ xn).reshape(s.n_kv_heads, dh)
             v = (self.W(w + "wv") @ xn).reshape(s.n_kv_heads, dh)
             q, k = rope(q, p, s.rope_theta), rope(k, p, s.rope_theta)
-            cache["K"][l, :, p, :] = k
-            cache["V"][l, :, p, :] = v
+            cache["K"][l, :, p, :] = self.kv(k)
+            cache["V"][l, :, p, :] = self.kv(v)
             o = attend_one(q, cache["K"][l, :, :p + 1, :], cache["V"][l, :, :p + 1, :])
             x = x + self.W(w + "wo") @ o.reshape(-1)
             xn = rmsnorm(x, self.w16[w + "mlp_norm"], s.rms_eps)

@@ -323,8 +323,8 @@ def test_zero_weight_closed_forms(which):
 
 def test_uniform_attention_layer_closed_form():
     # One layer, Wq = Wk = 0 (uniform weights over j <= p), Wv = Wo = I, FFN = 0:
-    # x_p' = x_p + mean_{j<=p} RMSNorm(x_j; g1). Pins causal masking, V and O paths
-    # and the residual add.
+    # x_p' = x_p + mean_{j<=p} fp16(RMSNorm(x_j; g1)) (V is cached in fp16). Pins
+    # causal masking, the V and O paths and the residual add.
     s = S.Shape("t-u", n_layers=1, d_model=8, n_heads=2, n_kv_heads=2, head_dim=4, ffn=4,
                 vocab=11, max_ctx=8)
     w = S.make_weights(s, seed=8, cache=False)
@@ -346,7 +346,7 @@ def test_uniform_attention_layer_closed_form():
         return np.array([v[i] / r * g[i] for i in range(len(v))])
 
     for p in range(5):
-        mean = sum(nrm(xs[j], g1) for j in range(p + 1)) / (p + 1)
+        mean = sum(nrm(xs[j], g1).astype(np.float16).astype(np.float64) for j in range(p + 1)) / (p + 1)
         xp = xs[p] + mean
         want = np.zeros(11); want[:8] = nrm(xp, np.ones(8))
         assert np.allclose(full[p], want, atol=1e-12)
@@ -361,3 +361,32 @@ def test_long_context_weights_are_prefix_of_dense():
     assert np.array_equal(w4["layers.0.wk"], w3["layers.0.wk"][:1024])
     assert np.array_equal(w4["layers.0.wv"], w3["layers.0.wv"][:1024])
     assert np.array_equal(w4["layers.0.wq"], w3["layers.0.wq"])
+
+
+def test_kv_cache_holds_fp16_rounded_values():
+    # The cache keeps K (after RoPE) and V rounded to fp16; queries are not rounded.
+    s = _tiny("gqa")
+    w = _scaled(S.make_weights(s, seed=11, cache=False), 10.0)
+    m = O.Decoder(s, w)
+    cache = m.new_cache(4)
+    toks = S.make_tokens(s, 3, seed=12)
+    for t in toks:
+        m.step(t, cache)
+    K, V = cache["K"][:, :, :3, :], cache["V"][:, :, :3, :]
+    assert np.array_equal(K.astype(np.float16).astype(np.float64), K)
+    assert np.array_equal(V.astype(np.float16).astype(np.float64), V)
+    # layer 0, position 0: v = Wv . RMSNorm(E[t0]) rounded to fp16 (elementwise, brute force)
+    e = w["embed"][toks[0]].astype(np.float64)
+    r = math.sqrt(sum(x * x for x in e) / len(e) + s.rms_eps)
+    g = w["layers.0.attn_norm"].astype(np.float64)
+    xn = [e[i] / r * g[i] for i in range(len(e))]
+    Wv = w["layers.0.wv"].astype(np.float64)
+    for row in range(Wv.shape[0]):
+        val = sum(Wv[row, j] * xn[j] for j in range(len(xn)))
+        assert V[0, row // s.head_dim, 0, row % s.head_dim] == float(np.float16(val))
+    # the unrounded variant differs (the rounding is really applied)
+    m2 = O.Decoder(s, w, kv_fp16=False)
+    c2 = m2.new_cache(4)
+    for t in toks:
+        m2.step(t, c2)
+    assert not np.array_equal(c2["V"][:, :, :3, :], V)
