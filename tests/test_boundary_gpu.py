@@ -218,5 +218,5 @@ def test_info_counts(eng):
     mats = L * (4 * d * d + 3 * ff * d) * 2 + V * d * 2
     assert info["stream_bytes"] == mats + (2 * L + 1) * d * 2 + d * 2
     assert info["kv_bytes_per_pos"] == 2 * L * SH.n_kv_heads * SH.head_dim * 2
-    assert info["grid"] >= 100 and info["threads"] == 288
+    assert info["grid"] >= 100 and info["threads"] == 256
     assert info["resident_bytes"] == mats

@@ -24,7 +24,7 @@
 #include "kie_internal.h"
 
 namespace kie {
-int kernel_smem_bytes(int vec_floats, int n_stages);
+int kernel_smem_bytes(int vec_floats, int n_stages, int stage_bytes);
 int kernel_max_stages();
 const void* kernel_entry();
 }  // namespace kie
@@ -43,6 +43,7 @@ struct kie_ctx {
   int sms = 0;
   int grid = 0;
   int n_stages = 0;
+  int stage_bytes = 0;
   int vec_floats = 0;
   int smem = 0;
   int max_chunks = 0;
@@ -129,13 +130,13 @@ bool is_device_ptr(const void* p) {
 // Tile shape for a segment kind: rows per tile g and column chunks nk. Prefer
 // g >= 4 (the input vector chunk is reused across g rows) with the fewest
 // chunks; GU kinds need an even g so (gate, up) pairs share a tile.
-SegShape choose_shape(int K, bool pairs) {
+SegShape choose_shape(int K, bool pairs, int stage_bytes) {
   SegShape best{K, 0, 0, 0};
   for (int nk = 1; nk <= 64; ++nk) {
     if (K % nk) continue;
     const int kc = K / nk;
     if (kc % 8) continue;
-    int g = std::min(kMaxRowsPerTile, kStageBytes / (2 * kc));
+    int g = std::min(kMaxRowsPerTile, stage_bytes / (2 * kc));
     if (pairs) g &= ~1;
     if (g < 1) continue;
     if (g >= 4) return SegShape{K, g, nk, kc};
@@ -144,7 +145,11 @@ SegShape choose_shape(int K, bool pairs) {
   return best;
 }
 
-int seg_rows_per_unit(int kind) { return (kind == SK_GU || kind == SK_SGU || kind == SK_EGU) ? 2 : 1; }
+// Rows are handed to CTAs in units: (gate, up) pairs for the FFN kinds and
+// RoPE pairs (dims i, i + dh/2 of one head) for q/k/v.
+int seg_rows_per_unit(int kind) {
+  return (kind == SK_GU || kind == SK_SGU || kind == SK_EGU || kind == SK_QKV) ? 2 : 1;
+}
 
 struct Tensor {
   const void* data;
@@ -265,16 +270,22 @@ kie_status kie_create(const kie_config* cfg, int device, kie_ctx** out) {
 
   const int hq = k.n_heads, hk = k.n_kv_heads, dh = k.head_dim, d = k.d_model;
   c->hbuf = moe ? (k.ffn_shared + k.top_k * k.ffn_expert) : k.ffn;
-  int vf = std::max({d, hq * dh, c->hbuf, kConsumerWarps * kMaxHeadsPerGroup * dh});
+  // the vector buffer doubles as attention scratch: q of one KV group, the
+  // consumer warps' (max, sum, acc) partials and their 32-position score blocks
+  int vf = std::max({d, hq * dh, c->hbuf,
+                     kMaxHeadsPerGroup * dh + kConsumerWarps * kMaxHeadsPerGroup * (dh + 4 + kAttnSub)});
   vf = (vf + 3) & ~3;
   c->vec_floats = vf;
-  const int fixed = kernel_smem_bytes(vf, 0);
+  // kRingStages ring stages (two per consumer warp) of the largest size that
+  // fits, in 1 KiB steps, at most 16 KiB
+  const int fixed = kernel_smem_bytes(vf, 0, 0);
   const int optin = (int)prop.sharedMemPerBlockOptin;
-  int ns = (optin - fixed) / kStageBytes;
-  ns = std::min(ns, kernel_max_stages());
-  if (ns < 3) return bail(fail(c, KIE_ERR_INVALID_ARG, "shape needs too much shared memory"));
+  const int ns = kernel_max_stages();
+  int sb = std::min(kMaxStageBytes, ((optin - fixed) / ns) & ~1023);
+  if (sb < 4096) return bail(fail(c, KIE_ERR_INVALID_ARG, "shape needs too much shared memory"));
   c->n_stages = ns;
-  c->smem = kernel_smem_bytes(vf, ns);
+  c->stage_bytes = sb;
+  c->smem = kernel_smem_bytes(vf, ns, sb);
   if (cudaFuncSetAttribute(kernel_entry(), cudaFuncAttributeMaxDynamicSharedMemorySize, c->smem) !=
       cudaSuccess)
     return bail(fail(c, KIE_ERR_CUDA, "cudaFuncSetAttribute(smem=%d) failed: %s", c->smem,
@@ -287,8 +298,9 @@ kie_status kie_create(const kie_config* cfg, int device, kie_ctx** out) {
   c->grid = c->sms;  // one CTA per SM; the ring takes the SM's shared memory
   c->slots = slots_per_layer(moe ? k.n_experts : 0);
 
-  const int nwarps = c->grid * kConsumerWarps;
-  c->max_chunks = std::min((k.max_ctx + kAttnSub - 1) / kAttnSub, nwarps / hk + 2);
+  // attention units cover >= 256 positions and >= T*hk/grid positions each
+  const int unit_min = kConsumerWarps * kAttnSub;
+  c->max_chunks = std::min((k.max_ctx + unit_min - 1) / unit_min, c->grid / hk + 2);
 
   kie_status s;
   const size_t kv = (size_t)k.n_layers * hk * k.max_ctx * dh * sizeof(__half);
@@ -371,7 +383,7 @@ kie_status kie_get_info(const kie_ctx* c, kie_info* info) {
   info->grid = c->grid;
   info->threads = kThreads;
   info->n_stages = c->n_stages;
-  info->stage_bytes = kStageBytes;
+  info->stage_bytes = c->stage_bytes;
   info->smem_bytes = c->smem;
   info->barriers_per_token = 5 * k.n_layers + 1;
   info->stream_bytes = c->stream_bytes;
@@ -484,17 +496,17 @@ kie_status kie_load_weights(kie_ctx* c, const kie_tensor* tensors, int n, void* 
 
   // segment shapes
   const int ffs = k.ffn_shared, ffe = k.ffn_expert;
-  c->shp[SK_QKV] = choose_shape(d, false);
-  c->shp[SK_O] = choose_shape(hq * dh, false);
-  c->shp[SK_LM] = choose_shape(d, false);
+  c->shp[SK_QKV] = choose_shape(d, false, c->stage_bytes);
+  c->shp[SK_O] = choose_shape(hq * dh, false, c->stage_bytes);
+  c->shp[SK_LM] = choose_shape(d, false, c->stage_bytes);
   if (!moe) {
-    c->shp[SK_GU] = choose_shape(d, true);
-    c->shp[SK_DOWN] = choose_shape(k.ffn, false);
+    c->shp[SK_GU] = choose_shape(d, true, c->stage_bytes);
+    c->shp[SK_DOWN] = choose_shape(k.ffn, false, c->stage_bytes);
   } else {
-    c->shp[SK_SGU] = choose_shape(d, true);
-    c->shp[SK_EGU] = choose_shape(d, true);
-    c->shp[SK_SDOWN] = choose_shape(ffs, false);
-    c->shp[SK_EDOWN] = choose_shape(ffe, false);
+    c->shp[SK_SGU] = choose_shape(d, true, c->stage_bytes);
+    c->shp[SK_EGU] = choose_shape(d, true, c->stage_bytes);
+    c->shp[SK_SDOWN] = choose_shape(ffs, false, c->stage_bytes);
+    c->shp[SK_EDOWN] = choose_shape(ffe, false, c->stage_bytes);
   }
 
   // row assignment
@@ -581,10 +593,14 @@ kie_status kie_load_weights(kie_ctx* c, const kie_tensor* tensors, int n, void* 
     const int kind = kind_of(l, slot);
     const std::string p = "layers." + std::to_string(l) + ".";
     switch (kind) {
-      case SK_QKV:
-        if (row < hq * dh) return dptr[p + "wq"] + (size_t)row * d * 2;
-        if (row < (hq + hk) * dh) return dptr[p + "wk"] + (size_t)(row - hq * dh) * d * 2;
-        return dptr[p + "wv"] + (size_t)(row - (hq + hk) * dh) * d * 2;
+      case SK_QKV: {
+        // virtual rows of a head run (0, dh/2, 1, dh/2 + 1, ...) so RoPE pairs are adjacent
+        const int H = row / dh, v = row % dh;
+        const int dim = (v & 1) ? v / 2 + dh / 2 : v / 2;
+        if (H < hq) return dptr[p + "wq"] + ((size_t)H * dh + dim) * d * 2;
+        if (H < hq + hk) return dptr[p + "wk"] + ((size_t)(H - hq) * dh + dim) * d * 2;
+        return dptr[p + "wv"] + ((size_t)(H - hq - hk) * dh + dim) * d * 2;
+      }
       case SK_O: return dptr[p + "wo"] + (size_t)row * hq * dh * 2;
       case SK_GU: return dptr[p + ((row & 1) ? "w_up" : "w_gate")] + (size_t)(row / 2) * d * 2;
       case SK_DOWN: return dptr[p + "w_down"] + (size_t)row * k.ffn * 2;
@@ -747,7 +763,7 @@ kie_status launch(kie_ctx* c, const Run& r, cudaStream_t st) {
   P.timeout_ns = (unsigned long long)(r.timeout_ms ? r.timeout_ms : 1000u) * 1000000ull;
   P.fault_cta = r.fault_cta; P.fault_barrier = r.fault_barrier;
   P.trace = reinterpret_cast<unsigned long long*>(r.trace); P.trace_cap = r.trace_cap;
-  P.n_stages = c->n_stages; P.vec_floats = c->vec_floats;
+  P.n_stages = c->n_stages; P.stage_bytes = c->stage_bytes; P.vec_floats = c->vec_floats;
 
   CUDA_TRY(c, cudaMemsetAsync(c->syncblk, 0, c->syncblk_bytes, st));
   void* args[] = {&P};

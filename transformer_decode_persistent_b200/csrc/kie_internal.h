@@ -8,12 +8,16 @@
 namespace kie {
 
 // ---- launch geometry ------------------------------------------------------
-constexpr int kConsumerWarps = 8;                      // GEMV / attention warps
+// 7 consumer warps + 1 producer warp = 256 threads: registers are allocated to
+// a CTA in 4-warp steps, so 8 warps keep the 255-register ceiling that the
+// attention sub-block loop needs (9 warps would be capped at 168 and spill).
+constexpr int kConsumerWarps = 7;                      // GEMV / attention warps
 constexpr int kConsumerThreads = kConsumerWarps * 32;  // named barrier 1 spans these
 constexpr int kThreads = kConsumerThreads + 32;        // + one producer (TMA) warp
-constexpr int kStageBytes = 16384;                     // one ring stage = one weight tile
+constexpr int kRingStages = 2 * kConsumerWarps;        // ring stages per CTA (2 per consumer warp)
+constexpr int kMaxStageBytes = 16384;                  // upper bound of one stage (one weight tile)
 constexpr int kMaxRowsPerTile = 8;                     // rows of one tile (register-blocked)
-constexpr int kPartFloats = 2048;                      // per-CTA partial-sum slots per phase
+constexpr int kPartFloats = 1024;                      // per-CTA partial-sum slots per phase
 constexpr int kMaxHeadsPerGroup = 4;                   // query heads per KV head (GQA)
 constexpr int kMaxTopK = 4;                            // routed experts per token
 constexpr int kAttnSub = 32;                           // positions per attention sub-block
@@ -116,7 +120,8 @@ struct Params {
   int fault_cta, fault_barrier;
   unsigned long long* trace; // device [grid][trace_cap][2] or null
   int trace_cap;
-  int n_stages;
+  int n_stages;     // multiple of kConsumerWarps: stage s belongs to warp s % kConsumerWarps
+  int stage_bytes;
   int vec_floats;
 };
 

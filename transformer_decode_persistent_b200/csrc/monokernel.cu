@@ -37,21 +37,24 @@
 
 namespace kie {
 
-constexpr int kMaxStages = 16;
+constexpr int kMaxStages = kRingStages;
 constexpr int kErrTimeout = -5;  // KIE_ERR_TIMEOUT
 constexpr int kErrDevice = -6;   // KIE_ERR_DEVICE
+
+constexpr int kRouteRing = 8;  // routing decisions kept for lagging issuer lanes
 
 struct SmemCtl {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
-  uint64_t route_bar;
   volatile int abort;
+  volatile unsigned route_seq;  // routing decisions published so far
   int tok;
   float margin;
-  int route_e[kMaxTopK];
+  int route_e[kRouteRing][kMaxTopK];
   float route_w[kMaxTopK];
   float red[64];
   Cand wcand[kConsumerWarps];
+  unsigned bcast;
 };
 
 // Shared-memory layout, identical on host and device.
@@ -60,8 +63,8 @@ __host__ __device__ inline int smem_ring_offset(int vec_floats) {
   int b = smem_ctl_bytes() + kPartFloats * 4 + vec_floats * 4;
   return (b + 1023) & ~1023;
 }
-__host__ __device__ inline int smem_total(int vec_floats, int n_stages) {
-  return smem_ring_offset(vec_floats) + n_stages * kStageBytes;
+__host__ __device__ inline int smem_total(int vec_floats, int n_stages, int stage_bytes) {
+  return smem_ring_offset(vec_floats) + n_stages * stage_bytes;
 }
 
 // ---------------------------------------------------------------- primitives
@@ -89,6 +92,18 @@ __device__ __forceinline__ bool mbar_test(uint64_t* b, unsigned parity) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(su32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// non-blocking probe of an mbarrier phase (never suspends the thread)
+__device__ __forceinline__ bool mbar_probe(uint64_t* b, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(su32(b)), "r"(parity)
@@ -131,6 +146,34 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
+// two packed fp16 values (by value, so register arrays stay in registers)
+__device__ __forceinline__ float2 h2f2(unsigned u) {
+  __half2 h;
+  memcpy(&h, &u, sizeof(h));
+  return __half22float2(h);
+}
+
+// Explicit shared-memory loads by 32-bit shared address: the ring and the
+// input vector are reached through pointers kept in the consumer's state, and
+// generic loads of shared memory are slower than ld.shared.
+__device__ __forceinline__ uint4 lds_u4(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float lds_f32(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts_f32(uint32_t a, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+__device__ __forceinline__ float4 lds_f4(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+  return v;
+}
 
 // 8 fp16 weights (one 16-byte chunk) against 8 fp32 inputs, accumulated in fp32.
 __device__ __forceinline__ float dot8(const uint4& w, const float4& a, const float4& b, float acc) {
@@ -171,6 +214,46 @@ __device__ __forceinline__ void cand_warp_merge(float& v1, int& i1, float& v2) {
   }
 }
 
+// Butterfly transpose-reduction: lane l holds v[j] = its share of the dot
+// product of position j; afterwards v[0] of lane l is the full sum for j = l.
+__device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const bool up = lane & 16;
+    const float send = up ? v[k] : v[k + 16];
+    const float keep = up ? v[k + 16] : v[k];
+    v[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const bool up = lane & 8;
+    const float send = up ? v[k] : v[k + 8];
+    const float keep = up ? v[k + 8] : v[k];
+    v[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const bool up = lane & 4;
+    const float send = up ? v[k] : v[k + 4];
+    const float keep = up ? v[k + 4] : v[k];
+    v[k] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const bool up = lane & 2;
+    const float send = up ? v[k] : v[k + 2];
+    const float keep = up ? v[k + 2] : v[k];
+    v[k] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+  }
+  {
+    const bool up = lane & 1;
+    const float send = up ? v[0] : v[1];
+    const float keep = up ? v[1] : v[0];
+    v[0] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+  }
+  return v[0];
+}
+
 // ---------------------------------------------------------------- errors
 
 __device__ void record_error(const Params& P, int code, int where, int step) {
@@ -184,13 +267,16 @@ __device__ void record_error(const Params& P, int code, int where, int step) {
 }
 
 // Bounded wait on an mbarrier phase. Returns false on abort or deadline.
+// `spin` waits with non-suspending probes: the producer's issuer lanes share
+// one warp and wait on different stages, and a lane suspended in try_wait
+// would hold up the others.
 __device__ bool wait_bar(const Params& P, SmemCtl* sc, uint64_t* b, unsigned parity, int where,
-                         int step) {
-  if (mbar_test(b, parity)) return true;
+                         int step, bool spin = false) {
+  if (spin ? mbar_probe(b, parity) : mbar_test(b, parity)) return true;
   const unsigned long long t0 = gtimer();
   for (unsigned it = 1;; ++it) {
-    if (mbar_test(b, parity)) return true;
-    if ((it & 7) == 0) {
+    if (spin ? mbar_probe(b, parity) : mbar_test(b, parity)) return true;
+    if ((it & 63) == 0) {
       if (sc->abort || ld_relaxed(&P.ctrl->abort)) {
         sc->abort = 1;
         return false;
@@ -204,37 +290,123 @@ __device__ bool wait_bar(const Params& P, SmemCtl* sc, uint64_t* b, unsigned par
   }
 }
 
+// ---------------------------------------------------------------- attention plan
+// Attention work for one layer at position pos (T = pos + 1 keys): units are
+// (KV head g, chunk of `per` positions), unit u handled by CTA u % grid; each
+// of the kConsumerWarps warps of a unit takes pw = per / kConsumerWarps
+// positions as nsb sub-blocks of 32. The K and V rows of every sub-block are
+// streamed through the ring like weight tiles: per (unit, sub-block round) the
+// ring carries 7 K tiles (sub-ranges 0..6) and then 7 V tiles, so that both
+// tiles of sub-range k land on the same consumer warp. The row of `pos` itself
+// is written during this step and is never in a tile; the warp that owns it
+// reads it directly.
+struct AttnPlan {
+  int T, per, pw, nsb, nchk, units;
+};
+__device__ __forceinline__ AttnPlan attn_plan(int pos, int hk, int grid) {
+  constexpr int kUnitMin = kConsumerWarps * kAttnSub;
+  AttnPlan a;
+  a.T = pos + 1;
+  int per = (int)(((long long)a.T * hk + grid - 1) / grid);
+  per = ((max(per, kUnitMin) + kUnitMin - 1) / kUnitMin) * kUnitMin;
+  a.per = per;
+  a.pw = per / kConsumerWarps;
+  a.nsb = a.pw / kAttnSub;
+  a.nchk = (a.T + per - 1) / per;
+  a.units = hk * a.nchk;
+  return a;
+}
+__device__ __forceinline__ int attn_units_of(const AttnPlan& a, int cta, int grid) {
+  return a.units > cta ? (a.units - cta + grid - 1) / grid : 0;
+}
+constexpr int kAttnTilesPerRound = 2 * kConsumerWarps;
+
 // ---------------------------------------------------------------- producer
 
 struct Producer {
+  // Each of the producer warp's lanes 0..n_stages-1 owns one ring stage and
+  // issues the bulk copies of the tiles that land in it (tile t -> stage
+  // t % n_stages). A bulk copy occupies its issuing thread for roughly one
+  // memory round trip, so one issuer per stage keeps n_stages copies in flight.
   const Params& P;
   SmemCtl* sc;
   unsigned char* ring;
   unsigned long long pol;
-  unsigned t = 0;  // tiles issued
+  const int lane;
+  unsigned t = 0;     // tiles walked (all lanes walk the same sequence)
+  unsigned mine = 0;  // tiles issued by this lane
   int step = 0;
 
-  __device__ Producer(const Params& p, SmemCtl* s, unsigned char* r) : P(p), sc(s), ring(r) {
+  __device__ Producer(const Params& p, SmemCtl* s, unsigned char* r, int ln)
+      : P(p), sc(s), ring(r), lane(ln) {
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  }
+
+  // Put tile tt (bytes at src; 0 bytes = an empty tile) into this lane's stage.
+  __device__ bool put(unsigned tt, const void* src, unsigned bytes) {
+    const unsigned n = tt / P.n_stages;
+    if (n > 0 && !wait_bar(P, sc, &sc->empty[lane], (n - 1) & 1u, 3, step)) return false;
+    mbar_expect_tx(&sc->full[lane], bytes);  // with 0 bytes this arrival completes the phase
+    if (bytes) bulk_g2s(ring + (size_t)lane * P.stage_bytes, src, bytes, &sc->full[lane], pol);
+    ++mine;
+    return true;
   }
 
   __device__ bool issue(const SegDesc& sd, const SegShape& sh) {
     const int ngroups = (sd.nrows + sh.g - 1) / sh.g;
-    const unsigned char* base = P.tape + sd.off;
+    const int ntiles = ngroups * sh.nk;
     const int ns = P.n_stages;
-    for (int gi = 0; gi < ngroups; ++gi) {
+    const unsigned char* base = P.tape + sd.off;
+    // first tile of this segment that lands in this lane's stage
+    for (int i = (int)((lane + ns - (int)(t % ns)) % ns); i < ntiles; i += ns) {
+      const int gi = i / sh.nk, kj = i - gi * sh.nk;
       const int gp = min(sh.g, sd.nrows - gi * sh.g);
       const unsigned bytes = (unsigned)gp * sh.kc * 2u;
-      const unsigned char* gsrc = base + (size_t)gi * sh.g * sh.K * 2;
-      for (int kj = 0; kj < sh.nk; ++kj) {
-        const int s = (int)(t % ns);
-        const unsigned n = t / ns;
-        if (n > 0 && !wait_bar(P, sc, &sc->empty[s], (n - 1) & 1u, 3, step)) return false;
-        mbar_expect_tx(&sc->full[s], bytes);
-        bulk_g2s(ring + (size_t)s * kStageBytes, gsrc + (size_t)kj * bytes, bytes, &sc->full[s], pol);
-        ++t;
+      if (!put(t + i, base + (size_t)gi * sh.g * sh.K * 2 + (size_t)kj * bytes, bytes)) return false;
+    }
+    t += ntiles;
+    return true;
+  }
+
+  // K/V rows of this CTA's attention units of layer l (see attn_plan).
+  __device__ bool issue_attn(int l, int pos) {
+    const int G = gridDim.x, ns = P.n_stages, hk = P.hk, dh = P.dh;
+    const AttnPlan ap = attn_plan(pos, hk, G);
+    const int nu = attn_units_of(ap, blockIdx.x, G);
+    const int per_unit = ap.nsb * kAttnTilesPerRound;
+    const int ntiles = nu * per_unit;
+    for (int i = (int)((lane + ns - (int)(t % ns)) % ns); i < ntiles; i += ns) {
+      const int uo = i / per_unit, r = i - uo * per_unit;
+      const int b = r / kAttnTilesPerRound, ti = r - b * kAttnTilesPerRound;
+      const int k = ti % kConsumerWarps;
+      const bool isv = ti >= kConsumerWarps;
+      const int u = blockIdx.x + uo * G;
+      const int g = u / ap.nchk, ch = u - g * ap.nchk;
+      const int j0 = ch * ap.per, j1 = min(ap.T, j0 + ap.per);
+      const int wj0 = j0 + k * ap.pw, wj1 = min(j1, wj0 + ap.pw);
+      const int jb = wj0 + b * kAttnSub;
+      const int rows = max(0, min(min(jb + kAttnSub, wj1), pos) - jb);
+      const __half* cache = (isv ? P.vcache : P.kcache) + ((size_t)(l * hk + g) * P.max_ctx + jb) * dh;
+      if (!put(t + i, cache, (unsigned)rows * dh * 2u)) return false;
+    }
+    t += ntiles;
+    return true;
+  }
+
+  // Spin until the consumers have published routing decision `round`.
+  __device__ bool wait_route(unsigned round) {
+    const unsigned long long t0 = gtimer();
+    for (unsigned it = 0; sc->route_seq <= round; ++it) {
+      if ((it & 63) == 63) {
+        if (sc->abort || ld_relaxed(&P.ctrl->abort)) return false;
+        if (gtimer() - t0 > P.timeout_ns) {
+          record_error(P, kErrTimeout, 4, step);
+          sc->abort = 1;
+          return false;
+        }
       }
     }
+    __threadfence_block();
     return true;
   }
 
@@ -246,7 +418,7 @@ struct Producer {
     for (step = 0; ok && step < P.n_steps; ++step) {
       for (int l = 0; ok && l < P.L; ++l) {
         const SegDesc* Dl = D + (size_t)l * P.slots;
-        ok = issue(Dl[0], P.shp[SK_QKV]) && issue(Dl[1], P.shp[SK_O]);
+        ok = issue(Dl[0], P.shp[SK_QKV]) && issue_attn(l, P.pos0 + step) && issue(Dl[1], P.shp[SK_O]);
         if (!ok) break;
         if (P.E == 0) {
           ok = issue(Dl[2], P.shp[SK_GU]) && issue(Dl[3], P.shp[SK_DOWN]);
@@ -254,11 +426,11 @@ struct Producer {
           ok = issue(Dl[2], P.shp[SK_SGU]);
           if (!ok) break;
           // the routed experts are known only once the consumers have run the router
-          ok = wait_bar(P, sc, &sc->route_bar, route_round & 1u, 4, step);
-          ++route_round;
+          ok = wait_route(route_round);
           if (!ok) break;
           int e[kMaxTopK];
-          for (int k = 0; k < P.top_k; ++k) e[k] = sc->route_e[k];
+          for (int k = 0; k < P.top_k; ++k) e[k] = sc->route_e[route_round % kRouteRing][k];
+          ++route_round;
           for (int k = 0; ok && k < P.top_k; ++k) ok = issue(Dl[4 + e[k]], P.shp[SK_EGU]);
           ok = ok && issue(Dl[3], P.shp[SK_SDOWN]);
           for (int k = 0; ok && k < P.top_k; ++k) ok = issue(Dl[4 + P.E + e[k]], P.shp[SK_EDOWN]);
@@ -266,12 +438,11 @@ struct Producer {
       }
       if (ok && step >= P.lm_from_step) ok = issue(D[(size_t)P.L * P.slots], P.shp[SK_LM]);
     }
-    // let every copy still in flight land before the CTA may exit
-    const int ns = P.n_stages;
-    for (unsigned tt = (t > (unsigned)ns ? t - ns : 0u); tt < t; ++tt) {
-      const int s = (int)(tt % ns);
+    // let this lane's last copy land before the CTA may exit
+    if (mine > 0) {
+      const unsigned n = (mine - 1);  // round of the last tile in this stage
       const unsigned long long t0 = gtimer();
-      while (!mbar_test(&sc->full[s], (tt / ns) & 1u)) {
+      while (!mbar_test(&sc->full[lane], n & 1u)) {
         if (gtimer() - t0 > P.timeout_ns) break;
       }
     }
@@ -280,21 +451,22 @@ struct Producer {
 
 // ---------------------------------------------------------------- consumer
 
-// One tile: G rows x nch 16-byte chunks, row-major in the stage. Lane l takes
-// chunks l, l+32, ...; the input vector chunk is read once and reused for all
-// G rows. Writes the G row partial sums to part[prow(r)].
+// One tile: G rows x nch 16-byte chunks, row-major in the stage at shared
+// address w_s; the fp32 input slice at x_s. Lane l takes chunks l, l+32, ...;
+// the input chunk is read once and reused for all G rows. Writes the G row
+// partial sums to part[pidx0 + r * pstride].
 template <int G>
-__device__ __forceinline__ void tile_gemv(const uint4* __restrict__ w, const float4* __restrict__ xv,
-                                          int nch, int lane, float* part, int pidx0, int pstride) {
+__device__ __forceinline__ void tile_gemv(uint32_t w_s, uint32_t x_s, int nch, int lane, float* part,
+                                          int pidx0, int pstride) {
   float acc[G];
 #pragma unroll
   for (int r = 0; r < G; ++r) acc[r] = 0.f;
 #pragma unroll 2
   for (int c = lane; c < nch; c += 32) {
-    const float4 a = xv[2 * c];
-    const float4 b = xv[2 * c + 1];
+    const float4 a = lds_f4(x_s + c * 32);
+    const float4 b = lds_f4(x_s + c * 32 + 16);
 #pragma unroll
-    for (int r = 0; r < G; ++r) acc[r] = dot8(w[r * nch + c], a, b, acc[r]);
+    for (int r = 0; r < G; ++r) acc[r] = dot8(lds_u4(w_s + (uint32_t)(r * nch + c) * 16u), a, b, acc[r]);
   }
   __syncwarp();
 #pragma unroll
@@ -338,35 +510,36 @@ struct Consumer {
     cbar();
   }
 
-  // vec = RMSNorm(src) * gain, src either fp32 (residual) or an fp16 embedding row.
+  // vec = RMSNorm(src) * gain, src either fp32 (residual) or an fp16 embedding
+  // row. The (read-only) gain is prefetched into L1 alongside the source loads,
+  // so the scaling pass after the block reduction does not pay a second L2
+  // round trip.
   __device__ void load_norm(const float* srcf, const __half* srch, const __half* gain, int n) {
     float ss = 0.f;
-    if (srcf) {
-      for (int i = tid * 4; i < n; i += kConsumerThreads * 4) {
-        const float4 v = *reinterpret_cast<const float4*>(srcf + i);
-        *reinterpret_cast<float4*>(vec + i) = v;
-        ss = fmaf(v.x, v.x, ss);
-        ss = fmaf(v.y, v.y, ss);
-        ss = fmaf(v.z, v.z, ss);
-        ss = fmaf(v.w, v.w, ss);
+    for (int i = tid * 4; i < n; i += kConsumerThreads * 4) {
+      asm volatile("prefetch.global.L1 [%0];" ::"l"(gain + i));
+      float4 v;
+      if (srcf) {
+        v = *reinterpret_cast<const float4*>(srcf + i);
+      } else {
+        const uint2 raw = *reinterpret_cast<const uint2*>(srch + i);
+        const float2 lo = h2f2(raw.x), hi = h2f2(raw.y);
+        v = make_float4(lo.x, lo.y, hi.x, hi.y);
       }
-    } else {
-      for (int i = tid * 8; i < n; i += kConsumerThreads * 8) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(srch + i);
-        const __half2* hh = reinterpret_cast<const __half2*>(&raw);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 f = __half22float2(hh[k]);
-          vec[i + 2 * k] = f.x;
-          vec[i + 2 * k + 1] = f.y;
-          ss = fmaf(f.x, f.x, ss);
-          ss = fmaf(f.y, f.y, ss);
-        }
-      }
+      *reinterpret_cast<float4*>(vec + i) = v;
+      ss = fmaf(v.x, v.x, ss);
+      ss = fmaf(v.y, v.y, ss);
+      ss = fmaf(v.z, v.z, ss);
+      ss = fmaf(v.w, v.w, ss);
     }
     const float tot = block_sum(ss);
     const float inv = 1.0f / sqrtf(tot / (float)n + P.eps);
-    for (int i = tid; i < n; i += kConsumerThreads) vec[i] = vec[i] * inv * __half2float(gain[i]);
+    for (int i = tid * 4; i < n; i += kConsumerThreads * 4) {
+      const uint2 g = __ldg(reinterpret_cast<const uint2*>(gain + i));
+      const float2 g0 = h2f2(g.x), g1 = h2f2(g.y);
+      const float4 v = *reinterpret_cast<const float4*>(vec + i);
+      *reinterpret_cast<float4*>(vec + i) = make_float4(v.x * inv * g0.x, v.y * inv * g0.y, v.z * inv * g1.x, v.w * inv * g1.y);
+    }
     cbar();
   }
 
@@ -377,15 +550,20 @@ struct Consumer {
     const int ntiles = ngroups * sh.nk;
     const int ns = P.n_stages;
     const int nch = sh.kc / 8;
-    for (int i = warp; i < ntiles; i += kConsumerWarps) {
+    // Tile t (ring position) always goes to warp t % kConsumerWarps, and the
+    // stage count is a multiple of kConsumerWarps, so every stage is only ever
+    // used by one warp, in order: its parity waits can never see a phase two
+    // rounds old.
+    const int first = (int)((warp + kConsumerWarps - (int)(tbase % kConsumerWarps)) % kConsumerWarps);
+    for (int i = first; i < ntiles; i += kConsumerWarps) {
       if (sc->abort) break;
       const unsigned t = tbase + i;
       const int s = (int)(t % ns);
       if (!wait_bar(P, sc, &sc->full[s], (t / ns) & 1u, 2, step)) break;
       const int gi = i / sh.nk, kj = i - gi * sh.nk;
       const int gp = min(sh.g, sd.nrows - gi * sh.g);
-      const uint4* w = reinterpret_cast<const uint4*>(ring + (size_t)s * kStageBytes);
-      const float4* xv = reinterpret_cast<const float4*>(vseg + (size_t)kj * sh.kc);
+      const uint32_t w = su32(ring) + (uint32_t)(s * P.stage_bytes);
+      const uint32_t xv = su32(vseg) + (uint32_t)(kj * sh.kc) * 4u;
       const int p0 = pbase + gi * sh.g * pstride + kjbase + kj;
       // the stage is released inside tile_gemv's reduction (after __syncwarp)
       switch (gp) {
@@ -420,14 +598,13 @@ struct Consumer {
         atomicExch(&P.ctrl->abort, 1u);
       } else {
         const bool skip = ((int)blockIdx.x == P.fault_cta && (int)k == P.fault_barrier);
-        if (!skip) {
-          __threadfence();
-          red_release_add(&P.ctrl->arrive, 1u);
-        }
+        // the consumer barrier above orders this CTA's writes before thread 0's
+        // release; the release-add publishes them at GPU scope
+        if (!skip) red_release_add(&P.ctrl->arrive, 1u);
         const unsigned target = (k + 1) * gridDim.x;
         const unsigned long long t0 = gtimer();
         unsigned it = 0;
-        while (ld_acquire(&P.ctrl->arrive) < target) {
+        while (ld_relaxed(&P.ctrl->arrive) < target) {
           if ((++it & 15) == 0) {
             if (ld_relaxed(&P.ctrl->abort)) {
               ab = 1;
@@ -440,6 +617,7 @@ struct Consumer {
             }
           }
         }
+        asm volatile("fence.acq_rel.gpu;" ::: "memory");  // acquire the other CTAs' writes
       }
       if (P.trace && (int)k < P.trace_cap) {
         unsigned long long* tr = P.trace + ((size_t)blockIdx.x * P.trace_cap + k) * 2;
@@ -452,166 +630,321 @@ struct Consumer {
     return !sc->abort;
   }
 
-  // ---- attention: split-K over positions, units (kv head, chunk), one warp each
+  // One warp's share of one attention unit for a KV group of NH query heads:
+  // its sub-range [wj0, wj1) in 32-position sub-blocks whose K and V tiles come
+  // through the ring, with online softmax; the (max, sum, acc) partials of
+  // each head go to wp. NH is a template parameter so every head loop is
+  // unrolled exactly, keeping the code small.
+  template <int DH, int NH>
+  __device__ void attn_warp(const AttnPlan& ap, int uo, int vs, int wj0, int wj1, int pos, uint2 kpos,
+                            uint2 vpos, float* qs, float* wp, float* sbuf) {
+    constexpr int DPL = DH / 32;
+    constexpr int WS = DH + 4;
+    const int ns = P.n_stages;
+    const uint32_t ring_s = su32(ring);
+    const uint32_t ssm = su32(sbuf) + (uint32_t)(warp * kMaxHeadsPerGroup * kAttnSub) * 4u;
+    const uint32_t qsa = su32(qs) + (uint32_t)(lane * DPL) * 4u;
+    float m[NH], ls[NH], acc[NH][DPL], acc2[NH][DPL];
+#pragma unroll
+    for (int hh = 0; hh < NH; ++hh) {
+      m[hh] = -INFINITY;
+      ls[hh] = 0.f;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[hh][e] = acc2[hh][e] = 0.f;
+    }
+    for (int b = 0; b < ap.nsb; ++b) {
+      const unsigned tK = tbase + (unsigned)((uo * ap.nsb + b) * kAttnTilesPerRound + vs);
+      const unsigned tV = tK + kConsumerWarps;
+      const int sK = (int)(tK % ns), sV = (int)(tV % ns);
+      const int jb = wj0 + b * kAttnSub;
+      const int nj = max(0, min(kAttnSub, wj1 - jb));                  // valid keys in the sub-block
+      const int nsm = max(0, min(min(jb + kAttnSub, wj1), pos) - jb);  // of which in the tile
+      const bool valid = lane < nj;
+      if (!wait_bar(P, sc, &sc->full[sK], (tK / ns) & 1u, 2, step)) sc->abort = 1;
+      const bool work = nj > 0 && !sc->abort;
+      if (work) {
+        const uint32_t kt = ring_s + (uint32_t)(sK * P.stage_bytes) + (uint32_t)(lane * DPL * 2);
+#pragma unroll 1
+        for (int hh = 0; hh < NH; ++hh) {
+          float q[DPL];
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) q[e] = lds_f32(qsa + (uint32_t)(hh * DH + e) * 4u);
+          float part[kAttnSub];
+#pragma unroll
+          for (int jj = 0; jj < kAttnSub; ++jj) {
+            uint2 kr = make_uint2(0u, 0u);
+            if (jj < nsm) {
+              if constexpr (DPL == 4) asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(kr.x), "=r"(kr.y) : "r"(kt + jj * DH * 2) : "memory");
+              else asm("ld.shared.u32 %0, [%1];" : "=r"(kr.x) : "r"(kt + jj * DH * 2) : "memory");
+            } else if (jj == nsm && jj < nj) {
+              kr = kpos;
+            }
+            const float2 a = h2f2(kr.x);
+            float tt = q[0] * a.x;
+            tt = fmaf(q[1], a.y, tt);
+            if constexpr (DPL == 4) {
+              const float2 c2 = h2f2(kr.y);
+              tt = fmaf(q[2], c2.x, tt);
+              tt = fmaf(q[3], c2.y, tt);
+            }
+            part[jj] = tt;
+          }
+          const float a = transpose_reduce32(part, lane);
+          sts_f32(ssm + (uint32_t)(hh * kAttnSub + lane) * 4u, valid ? a : -INFINITY);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sc->empty[sK]);
+      if (!wait_bar(P, sc, &sc->full[sV], (tV / ns) & 1u, 2, step)) sc->abort = 1;
+      if (work && !sc->abort) {
+        float p[NH];
+#pragma unroll
+        for (int hh = 0; hh < NH; ++hh) {
+          const float sv = lds_f32(ssm + (uint32_t)(hh * kAttnSub + lane) * 4u);
+          const float mn = fmaxf(m[hh], warp_max(sv));
+          p[hh] = valid ? expf(sv - mn) : 0.f;
+          const float corr = expf(m[hh] - mn);
+          ls[hh] = ls[hh] * corr + warp_sum(p[hh]);
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) {
+            acc[hh][e] *= corr;
+            acc2[hh][e] *= corr;
+          }
+          m[hh] = mn;
+        }
+        const uint32_t vt = ring_s + (uint32_t)(sV * P.stage_bytes) + (uint32_t)(lane * DPL * 2);
+#pragma unroll 2
+        for (int jj = 0; jj < nj; jj += 2) {
+          uint2 va = make_uint2(0u, 0u), vb = make_uint2(0u, 0u);
+          if (jj < nsm) {
+            if constexpr (DPL == 4) asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(va.x), "=r"(va.y) : "r"(vt + jj * DH * 2) : "memory");
+            else asm("ld.shared.u32 %0, [%1];" : "=r"(va.x) : "r"(vt + jj * DH * 2) : "memory");
+          } else if (jj == nsm) {
+            va = vpos;
+          }
+          if (jj + 1 < nsm) {
+            if constexpr (DPL == 4) asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(vb.x), "=r"(vb.y) : "r"(vt + (jj + 1) * DH * 2) : "memory");
+            else asm("ld.shared.u32 %0, [%1];" : "=r"(vb.x) : "r"(vt + (jj + 1) * DH * 2) : "memory");
+          } else if (jj + 1 == nsm && jj + 1 < nj) {
+            vb = vpos;
+          }
+          float fa[DPL], fb[DPL];
+          {
+            const float2 a0 = h2f2(va.x), b0 = h2f2(vb.x);
+            fa[0] = a0.x; fa[1] = a0.y; fb[0] = b0.x; fb[1] = b0.y;
+            if constexpr (DPL == 4) {
+              const float2 a1 = h2f2(va.y), b1 = h2f2(vb.y);
+              fa[2] = a1.x; fa[3] = a1.y; fb[2] = b1.x; fb[3] = b1.y;
+            }
+          }
+#pragma unroll
+          for (int hh = 0; hh < NH; ++hh) {
+            const float pa = __shfl_sync(0xffffffffu, p[hh], jj);
+            const float pb = __shfl_sync(0xffffffffu, p[hh], (jj + 1) & 31);
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) {
+              acc[hh][e] = fmaf(pa, fa[e], acc[hh][e]);
+              acc2[hh][e] = fmaf(pb, fb[e], acc2[hh][e]);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sc->empty[sV]);
+    }
+    // partials -> shared memory (an empty range gives m = -inf, l = 0)
+#pragma unroll
+    for (int hh = 0; hh < NH; ++hh) {
+      float* pb = wp + (warp * kMaxHeadsPerGroup + hh) * WS;
+      if (lane == 0) {
+        pb[0] = m[hh];
+        pb[1] = ls[hh];
+      }
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) pb[4 + lane * DPL + e] = acc[hh][e] + acc2[hh][e];
+    }
+  }
+
+  // ---- attention over the KV cache (q already rotated and scaled; this
+  // token's k/v appended by the q/k/v epilogue). K and V rows arrive through
+  // the ring (see attn_plan); each warp handles one sub-range of each of the
+  // CTA's units, lanes over head dims for both q.k (butterfly transpose-reduce
+  // of 32 positions) and the V sum. The warps' (max, sum, acc) partials are
+  // merged in shared memory; a head spanning several CTAs is finished by the
+  // last of them (arrival counter per KV head) from per-CTA partials.
   template <int DH>
   __device__ void attention(int l, int pos) {
-    constexpr int DPL = DH / 32;  // dims per lane in the V accumulation
-    const int T = pos + 1;
-    const int hk = P.hk, hq = P.hq;
-    const int nwarps = gridDim.x * kConsumerWarps;
-    int pc = (T * hk + nwarps - 1) / nwarps;
-    pc = ((max(pc, kAttnSub) + kAttnSub - 1) / kAttnSub) * kAttnSub;
-    const int nch = (T + pc - 1) / pc;
-    const int units = hk * nch;
-    float* qs = vec + warp * (kMaxHeadsPerGroup * DH);
-    const float2* rp = P.rope + (size_t)pos * (DH / 2);
-    const float scale = rsqrtf((float)DH);
-    for (int u = blockIdx.x * kConsumerWarps + warp; u < units; u += nwarps) {
-      const int g = u / nch, ch = u - (u / nch) * nch;
+    constexpr int DPL = DH / 32;   // head dims per lane
+    constexpr int WS = DH + 4;     // partial record: m, l, pad, pad, acc[DH]
+    const int hk = P.hk, hq = P.hq, G = gridDim.x, ns = P.n_stages;
+    const AttnPlan ap = attn_plan(pos, hk, G);
+    const int nu = attn_units_of(ap, blockIdx.x, G);
+    const int vs = (int)((warp + kConsumerWarps - (int)(tbase % kConsumerWarps)) % kConsumerWarps);
+    float* qs = vec;                                              // [nh][DH]
+    float* wp = vec + kMaxHeadsPerGroup * DH;                     // [warp][hh][WS]
+    float* sbuf = wp + kConsumerWarps * kMaxHeadsPerGroup * WS;   // [warp][hh][32] scores
+    const uint32_t ring_s = su32(ring);
+    for (int uo = 0; uo < nu; ++uo) {
+      const int u = blockIdx.x + uo * G;
+      const int g = u / ap.nchk, ch = u - g * ap.nchk;
       const int h_lo = (g * hq + hk - 1) / hk;
       const int nh = (((g + 1) * hq + hk - 1) / hk) - h_lo;
-      // rotated, pre-scaled queries of the group's heads
-      for (int hh = 0; hh < nh; ++hh) {
-        const float* qr = P.qkv + (size_t)(h_lo + hh) * DH;
-        for (int i = lane; i < DH / 2; i += 32) {
-          const float a = qr[i], b = qr[i + DH / 2];
-          const float2 cs = rp[i];
-          qs[hh * DH + i] = (a * cs.x - b * cs.y) * scale;
-          qs[hh * DH + i + DH / 2] = (a * cs.y + b * cs.x) * scale;
+      const int j0 = ch * ap.per, j1 = min(ap.T, j0 + ap.per);
+      const int wj0 = j0 + vs * ap.pw, wj1 = min(j1, wj0 + ap.pw);
+      // this token's own row is not in the ring: fetch it now, use it last
+      uint2 kpos = make_uint2(0u, 0u), vpos = make_uint2(0u, 0u);
+      if (wj0 <= pos && pos < wj1) {
+        const size_t ro = ((size_t)(l * hk + g) * P.max_ctx + pos) * DH + lane * DPL;
+        if constexpr (DPL == 4) {
+          kpos = *reinterpret_cast<const uint2*>(P.kcache + ro);
+          vpos = *reinterpret_cast<const uint2*>(P.vcache + ro);
+        } else {
+          kpos.x = *reinterpret_cast<const unsigned*>(P.kcache + ro);
+          vpos.x = *reinterpret_cast<const unsigned*>(P.vcache + ro);
         }
       }
-      __half* Kc = P.kcache + ((size_t)(l * hk + g) * P.max_ctx) * DH;
-      __half* Vc = P.vcache + ((size_t)(l * hk + g) * P.max_ctx) * DH;
-      if (ch == nch - 1) {  // append this token's rotated k and its v at position pos
-        const float* kr = P.qkv + (size_t)hq * DH + (size_t)g * DH;
-        const float* vr = P.qkv + (size_t)(hq + hk) * DH + (size_t)g * DH;
-        for (int i = lane; i < DH / 2; i += 32) {
-          const float a = kr[i], b = kr[i + DH / 2];
-          const float2 cs = rp[i];
-          Kc[(size_t)pos * DH + i] = __float2half_rn(a * cs.x - b * cs.y);
-          Kc[(size_t)pos * DH + i + DH / 2] = __float2half_rn(a * cs.y + b * cs.x);
-          Vc[(size_t)pos * DH + i] = __float2half_rn(vr[i]);
-          Vc[(size_t)pos * DH + i + DH / 2] = __float2half_rn(vr[i + DH / 2]);
-        }
+      for (int i = tid; i < nh * DH; i += kConsumerThreads) qs[i] = P.qkv[(size_t)h_lo * DH + i];
+      cbar();
+      switch (nh) {
+        case 1: attn_warp<DH, 1>(ap, uo, vs, wj0, wj1, pos, kpos, vpos, qs, wp, sbuf); break;
+        case 2: attn_warp<DH, 2>(ap, uo, vs, wj0, wj1, pos, kpos, vpos, qs, wp, sbuf); break;
+        case 3: attn_warp<DH, 3>(ap, uo, vs, wj0, wj1, pos, kpos, vpos, qs, wp, sbuf); break;
+        default: attn_warp<DH, 4>(ap, uo, vs, wj0, wj1, pos, kpos, vpos, qs, wp, sbuf); break;
       }
-      __syncwarp();
-      const int j0 = ch * pc, j1 = min(T, j0 + pc);
-      float m[kMaxHeadsPerGroup], ls[kMaxHeadsPerGroup], acc[kMaxHeadsPerGroup][DPL];
+      cbar();
+      // merge the consumer warps' partials: warp hh merges head hh
+      if (warp < nh) {
+        const int hh = warp;
+        float M = -INFINITY;
 #pragma unroll
-      for (int hh = 0; hh < kMaxHeadsPerGroup; ++hh) {
-        m[hh] = -INFINITY;
-        ls[hh] = 0.f;
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, wp[(w * kMaxHeadsPerGroup + hh) * WS]);
+        float Ls = 0.f, a[DPL];
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) acc[hh][e] = 0.f;
-      }
-      for (int jb = j0; jb < j1; jb += kAttnSub) {
-        const int j = jb + lane;
-        const bool valid = j < j1;
-        float s[kMaxHeadsPerGroup];
+        for (int e = 0; e < DPL; ++e) a[e] = 0.f;
 #pragma unroll
-        for (int hh = 0; hh < kMaxHeadsPerGroup; ++hh) s[hh] = 0.f;
-        if (valid) {
-          const uint4* kr = reinterpret_cast<const uint4*>(Kc + (size_t)j * DH);
-          uint4 kv[DH / 8];
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float* pb = wp + (w * kMaxHeadsPerGroup + hh) * WS;
+          const float sc_w = expf(pb[0] - M);
+          Ls = fmaf(sc_w, pb[1], Ls);
 #pragma unroll
-          for (int i = 0; i < DH / 8; ++i) kv[i] = kr[i];
-#pragma unroll
-          for (int hh = 0; hh < kMaxHeadsPerGroup; ++hh) {
-            if (hh < nh) {
-              const float4* q4 = reinterpret_cast<const float4*>(qs + hh * DH);
-              float a = 0.f;
-#pragma unroll
-              for (int i = 0; i < DH / 8; ++i) a = dot8(kv[i], q4[2 * i], q4[2 * i + 1], a);
-              s[hh] = a;
-            }
-          }
+          for (int e = 0; e < DPL; ++e) a[e] = fmaf(sc_w, pb[4 + lane * DPL + e], a[e]);
         }
-        float p[kMaxHeadsPerGroup];
-#pragma unroll
-        for (int hh = 0; hh < kMaxHeadsPerGroup; ++hh) {
-          if (hh < nh) {
-            const float sv = valid ? s[hh] : -INFINITY;
-            const float mn = fmaxf(m[hh], warp_max(sv));
-            p[hh] = valid ? expf(sv - mn) : 0.f;
-            const float corr = expf(m[hh] - mn);
-            ls[hh] = ls[hh] * corr + warp_sum(p[hh]);
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) acc[hh][e] *= corr;
-            m[hh] = mn;
-          }
-        }
-        const int nj = min(kAttnSub, j1 - jb);
-#pragma unroll 4
-        for (int jj = 0; jj < nj; ++jj) {
-          const __half* vrow = Vc + (size_t)(jb + jj) * DH + lane * DPL;
-          float vv[DPL];
-          if constexpr (DPL == 4) {
-            const uint2 raw = *reinterpret_cast<const uint2*>(vrow);
-            const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-            const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-            vv[0] = a.x; vv[1] = a.y; vv[2] = b.x; vv[3] = b.y;
-          } else {
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) vv[e] = __half2float(vrow[e]);
-          }
-#pragma unroll
-          for (int hh = 0; hh < kMaxHeadsPerGroup; ++hh) {
-            if (hh < nh) {
-              const float pj = __shfl_sync(0xffffffffu, p[hh], jj);
-#pragma unroll
-              for (int e = 0; e < DPL; ++e) acc[hh][e] = fmaf(pj, vv[e], acc[hh][e]);
-            }
-          }
-        }
-      }
-      // partials (m, l, acc) of this chunk
-      const int stride = DH + 4;
-#pragma unroll
-      for (int hh = 0; hh < kMaxHeadsPerGroup; ++hh) {
-        if (hh < nh) {
-          float* pb = P.apart + ((size_t)(h_lo + hh) * P.max_chunks + ch) * stride;
-          if (lane == 0) {
-            pb[0] = m[hh];
-            pb[1] = ls[hh];
-          }
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) pb[4 + lane * DPL + e] = acc[hh][e];
-        }
-      }
-      __threadfence();
-      __syncwarp();
-      unsigned old = 0;
-      if (lane == 0) old = atomicAdd(&P.acnt[g], 1u);
-      old = __shfl_sync(0xffffffffu, old, 0);
-      if (old == (unsigned)(nch - 1)) {  // last chunk of this KV head: combine
-        __threadfence();
-        for (int hh = 0; hh < nh; ++hh) {
-          const float* hb = P.apart + (size_t)(h_lo + hh) * P.max_chunks * stride;
-          float M = -INFINITY;
-          for (int cc = lane; cc < nch; cc += 32) M = fmaxf(M, __ldcg(hb + (size_t)cc * stride));
-          M = warp_max(M);
-          float Ls = 0.f, a[DPL];
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) a[e] = 0.f;
-          for (int cc = 0; cc < nch; ++cc) {
-            const float* cb = hb + (size_t)cc * stride;
-            const float w = expf(__ldcg(cb) - M);
-            Ls = fmaf(w, __ldcg(cb + 1), Ls);
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) a[e] = fmaf(w, __ldcg(cb + 4 + lane * DPL + e), a[e]);
-          }
+        const int h = h_lo + hh;
+        if (ap.nchk == 1) {
           const float inv = 1.0f / Ls;
 #pragma unroll
-          for (int e = 0; e < DPL; ++e) P.o[(size_t)(h_lo + hh) * DH + lane * DPL + e] = a[e] * inv;
+          for (int e = 0; e < DPL; ++e) P.o[(size_t)h * DH + lane * DPL + e] = a[e] * inv;
+        } else {
+          float* gb = P.apart + ((size_t)h * P.max_chunks + ch) * WS;
+          if (lane == 0) {
+            gb[0] = M;
+            gb[1] = Ls;
+          }
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) gb[4 + lane * DPL + e] = a[e];
         }
-        if (lane == 0) P.acnt[g] = 0u;
       }
+      if (ap.nchk > 1) {
+        cbar();
+        if (tid == 0) {
+          unsigned old;
+          asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(P.acnt + g) : "memory");
+          sc->bcast = old;
+        }
+        cbar();
+        if (sc->bcast == (unsigned)(ap.nchk - 1)) {  // last CTA of this KV head: merge the chunks
+          if (warp < nh) {
+            const int h = h_lo + warp;
+            const int nchk = ap.nchk;
+            const float* hb = P.apart + (size_t)h * P.max_chunks * WS;
+            float M = -INFINITY;
+            for (int c = lane; c < nchk; c += 32) M = fmaxf(M, __ldcg(hb + (size_t)c * WS));
+            M = warp_max(M);
+            float Ls = 0.f, a[DPL];
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) a[e] = 0.f;
+            for (int c0 = 0; c0 < nchk; c0 += 32) {
+              const int nc = min(32, nchk - c0);
+              float wl = 0.f;
+              if (lane < nc) {
+                const float* cb = hb + (size_t)(c0 + lane) * WS;
+                wl = expf(__ldcg(cb) - M);
+                Ls = fmaf(wl, __ldcg(cb + 1), Ls);
+              }
+              for (int cb0 = 0; cb0 < nc; cb0 += 8) {
+                float4 v8[8];
+#pragma unroll
+                for (int uu = 0; uu < 8; ++uu) {
+                  const float* src = hb + (size_t)(c0 + cb0 + uu) * WS + 4 + lane * DPL;
+                  if (cb0 + uu < nc) {
+                    if constexpr (DPL == 4) v8[uu] = __ldcg(reinterpret_cast<const float4*>(src));
+                    else v8[uu] = make_float4(__ldcg(src), __ldcg(src + 1), 0.f, 0.f);
+                  } else {
+                    v8[uu] = make_float4(0.f, 0.f, 0.f, 0.f);
+                  }
+                }
+#pragma unroll
+                for (int uu = 0; uu < 8; ++uu) {
+                  const float w = __shfl_sync(0xffffffffu, wl, (cb0 + uu) & 31);
+                  a[0] = fmaf(w, v8[uu].x, a[0]);
+                  a[1] = fmaf(w, v8[uu].y, a[1]);
+                  if constexpr (DPL == 4) {
+                    a[2] = fmaf(w, v8[uu].z, a[2]);
+                    a[3] = fmaf(w, v8[uu].w, a[3]);
+                  }
+                }
+              }
+            }
+            Ls = warp_sum(Ls);
+            const float inv = 1.0f / Ls;
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) P.o[(size_t)h * DH + lane * DPL + e] = a[e] * inv;
+          }
+          if (tid == 0) P.acnt[g] = 0u;
+        }
+      }
+      cbar();  // qs / wp are reused by the next unit
     }
+    tbase += (unsigned)(nu * ap.nsb * kAttnTilesPerRound);
   }
 
   __device__ void attention_dispatch(int l, int pos) {
     if (P.dh == 128) attention<128>(l, pos);
     else attention<64>(l, pos);
+  }
+
+  // q/k/v epilogue. The q/k/v rows are packed so that every CTA owns whole
+  // RoPE pairs (dims i and i + dh/2 of one head are adjacent virtual rows), so
+  // RoPE is applied here: q is rotated and pre-scaled by 1/sqrt(dh) into the q
+  // scratch, k is rotated and appended (fp16) to the KV cache at `pos`, v is
+  // appended as is.
+  __device__ void epi_qkv(const SegDesc& sd, int stride, int l, int pos) {
+    const int dh = P.dh, half = P.dh / 2, hq = P.hq, hk = P.hk;
+    const float2* rp = P.rope + (size_t)pos * half;
+    const float scale = 1.0f / sqrtf((float)dh);
+    for (int j = tid; j < sd.nrows / 2; j += kConsumerThreads) {
+      const int r = sd.row0 + 2 * j;
+      const int H = r / dh, pi = (r - H * dh) / 2;
+      const float ya = row_sum(2 * j, stride), yb = row_sum(2 * j + 1, stride);
+      if (H < hq + hk) {
+        const float2 cs = rp[pi];
+        const float a = ya * cs.x - yb * cs.y, b = ya * cs.y + yb * cs.x;
+        if (H < hq) {
+          P.qkv[(size_t)H * dh + pi] = a * scale;
+          P.qkv[(size_t)H * dh + pi + half] = b * scale;
+        } else {
+          __half* k = P.kcache + ((size_t)(l * hk + (H - hq)) * P.max_ctx + pos) * dh;
+          k[pi] = __float2half_rn(a);
+          k[pi + half] = __float2half_rn(b);
+        }
+      } else {
+        __half* v = P.vcache + ((size_t)(l * hk + (H - hq - hk)) * P.max_ctx + pos) * dh;
+        v[pi] = __float2half_rn(ya);
+        v[pi + half] = __float2half_rn(yb);
+      }
+    }
+    // the cache rows written here are read by TMA (async proxy) in later steps
+    asm volatile("fence.proxy.async.global;" ::: "memory");
   }
 
   // residual epilogue: x[row] = xprev[row] + sum of partials
@@ -658,6 +991,7 @@ struct Consumer {
       for (int e = 0; e < P.E; ++e) pr[e] = expf(part[e] - mx);
       unsigned long long used = 0ull;
       float wsum = 0.f;
+      int* re = sc->route_e[route_round % kRouteRing];
       for (int k = 0; k < P.top_k; ++k) {
         int bi = -1;
         float bv = -INFINITY;
@@ -667,14 +1001,16 @@ struct Consumer {
             bv = pr[e];
           }
         used |= 1ull << bi;
-        sc->route_e[k] = bi;
+        re[k] = bi;
         sc->route_w[k] = bv;
         wsum += bv;
       }
       for (int k = 0; k < P.top_k; ++k) sc->route_w[k] /= wsum;
-      mbar_arrive(&sc->route_bar);  // hand the choice to the producer
+      __threadfence_block();
+      sc->route_seq = route_round + 1;  // hand the choice to the producer lanes
     }
     cbar();
+    ++route_round;
   }
 
   __device__ bool layer(int l, int tok, int pos, const SegDesc* D) {
@@ -686,7 +1022,7 @@ struct Consumer {
     const SegShape& sq = P.shp[SK_QKV];
     run_segment(Dl[0], sq, vec, 0, sq.nk, 0);
     cbar();
-    for (int r = tid; r < Dl[0].nrows; r += kConsumerThreads) P.qkv[Dl[0].row0 + r] = row_sum(r, sq.nk);
+    epi_qkv(Dl[0], sq.nk, l, pos);
     if (!grid_sync()) return false;
     // ---- RoPE, KV append, attention
     attention_dispatch(l, pos);
@@ -713,11 +1049,12 @@ struct Consumer {
       epi_residual(Dl[3], sd.nk, nullptr);
       if (!grid_sync()) return false;
     } else {
+      const int* re = sc->route_e[route_round % kRouteRing];
       route(l);
       int e[kMaxTopK];
       float w[kMaxTopK];
       for (int k = 0; k < P.top_k; ++k) {
-        e[k] = sc->route_e[k];
+        e[k] = re[k];
         w[k] = sc->route_w[k];
       }
       const SegShape& ss = P.shp[SK_SGU];
@@ -840,14 +1177,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       mbar_init(&sc->full[s], 1);
       mbar_init(&sc->empty[s], 1);
     }
-    mbar_init(&sc->route_bar, 1);
+    sc->route_seq = 0;
     sc->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
   if (threadIdx.x >= kConsumerThreads) {
-    if (threadIdx.x == kConsumerThreads) {
-      Producer pr(P, sc, ring);
+    const int lane = threadIdx.x - kConsumerThreads;
+    if (lane < P.n_stages) {
+      Producer pr(P, sc, ring, lane);
       pr.run();
     }
     return;
@@ -857,7 +1195,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 }
 
 // ---- host-side accessors used by the launcher
-int kernel_smem_bytes(int vec_floats, int n_stages) { return smem_total(vec_floats, n_stages); }
+int kernel_smem_bytes(int vec_floats, int n_stages, int stage_bytes) {
+  return smem_total(vec_floats, n_stages, stage_bytes);
+}
 int kernel_max_stages() { return kMaxStages; }
 const void* kernel_entry() { return reinterpret_cast<const void*>(&decode_kernel); }
 
