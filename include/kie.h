@@ -145,6 +145,28 @@ kie_status kie_prefill(kie_ctx* ctx, const int32_t* tokens, int n, void* stream)
 kie_status kie_decode(kie_ctx* ctx, int n_tokens, int32_t* out_tokens,
                       const kie_decode_opts* opts, void* stream);
 
+/* Decode `n_tokens` tokens like kie_decode (free-running greedy, one persistent
+ * launch), for callers that must not allocate device memory while they run:
+ * for example a serving loop with a latency budget that cannot stall on the
+ * driver's allocator (cudaMalloc may synchronise the device), or a component
+ * that runs where all device memory belongs to another framework's pool.
+ * There is no counterpart of this call in the paper; it is an integration aid.
+ *
+ * The call allocates nothing and frees nothing. The kernel's per-launch
+ * scratch lives in a 512 KiB array in the library's device image, which every
+ * GPU that loads the library holds until the process exits. Models whose
+ * scratch (about 4 bytes per residual, q/k/v, attention-output and FFN value,
+ * plus attention partials) exceeds it are rejected with KIE_ERR_INVALID_ARG
+ * and a message giving both sizes. `out_tokens` must be device memory
+ * ([n_tokens] int32, caller-owned); no logits, margins, forced tokens or trace.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture. Every call on every context of a device shares the one array:
+ * calls whose work overlaps on the GPU race and give wrong results; issue
+ * them one after another. Errors: as kie_decode, plus INVALID_ARG for a host
+ * `out_tokens` or a model whose scratch does not fit. */
+kie_status kie_decode_static(kie_ctx* ctx, int n_tokens, int32_t* out_tokens, void* stream);
+
 /* Truncate the sequence to its first `pos` committed positions (0 <= pos <=
  * current position) and make `pending` (in [0, vocab)) the token fed to the
  * next forward, e.g. to regenerate from a prefix. KV entries at positions >= pos

@@ -16,6 +16,7 @@
 #include <cstdio>
 #include <cstring>
 #include <map>
+#include <mutex>
 #include <new>
 #include <string>
 #include <vector>
@@ -915,3 +916,136 @@ kie_status kie_decode(kie_ctx* c, int n, int32_t* out_tokens, const kie_decode_o
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------ no-allocation decode
+//
+// kie_decode_static runs the same persistent decode kernel as kie_decode, but
+// the kernel's per-launch scratch (residual stream, q/k/v, attention output,
+// FFN hidden vector, attention partials and arrival counters, per-CTA argmax
+// candidates, control block) lives in this file-scope device array instead of
+// buffers allocated with the context. The call itself allocates nothing.
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = 512u << 10;  // 512 KiB per device
+constexpr int kMaxDevices = 64;
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+namespace {
+
+std::mutex g_static_mu;
+unsigned char* g_static_ptr[kMaxDevices] = {};
+
+size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+struct StaticLayout {
+  size_t x, qkv, o, h, apart, cand, sync, total;
+};
+
+StaticLayout static_layout(const kie_ctx* c) {
+  const kie_config& k = c->cfg;
+  StaticLayout L{};
+  size_t off = 0;
+  L.sync = off;  off += align256(sizeof(Ctrl) + (size_t)k.n_kv_heads * sizeof(unsigned));
+  L.x = off;     off += align256((size_t)k.d_model * 4);
+  L.qkv = off;   off += align256((size_t)(k.n_heads + 2 * k.n_kv_heads) * k.head_dim * 4);
+  L.o = off;     off += align256((size_t)k.n_heads * k.head_dim * 4);
+  L.h = off;     off += align256((size_t)c->hbuf * 4);
+  L.apart = off; off += align256((size_t)k.n_heads * c->max_chunks * (k.head_dim + 4) * 4);
+  L.cand = off;  off += align256((size_t)c->grid * sizeof(Cand));
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+extern "C" kie_status kie_decode_static(kie_ctx* c, int n, int32_t* out_tokens, void* stream) {
+  if (!c) return KIE_ERR_INVALID_ARG;
+  c->err.clear();
+  if (c->poisoned) return fail(c, KIE_ERR_STATE, "context is poisoned; call kie_reset");
+  if (!c->loaded) return fail(c, KIE_ERR_STATE, "weights not loaded");
+  const StaticLayout lay = static_layout(c);
+  if (lay.total > kStaticScratchBytes)
+    return fail(c, KIE_ERR_INVALID_ARG, "this model needs %zu bytes of scratch; the static area holds %zu",
+                lay.total, kStaticScratchBytes);
+  if (c->device < 0 || c->device >= kMaxDevices) return fail(c, KIE_ERR_INVALID_ARG, "device %d out of range", c->device);
+  if (n < 0) return fail(c, KIE_ERR_INVALID_ARG, "negative token count");
+  if (n == 0) return KIE_OK;
+  if (!out_tokens || !is_device_ptr(out_tokens))
+    return fail(c, KIE_ERR_INVALID_ARG, "out_tokens must be device memory");
+  if (c->pending < 0) return fail(c, KIE_ERR_STATE, "no pending token: prefill first");
+  if ((int64_t)c->pos + n > c->cfg.max_ctx)
+    return fail(c, KIE_ERR_CONTEXT_FULL, "position %d + %d tokens exceeds max_ctx %d", c->pos, n, c->cfg.max_ctx);
+  CUDA_TRY(c, cudaSetDevice(c->device));
+  unsigned char* base = nullptr;
+  {
+    // once per device, with that device current: the array's device address
+    std::lock_guard<std::mutex> g(g_static_mu);
+    if (!g_static_ptr[c->device]) {
+      void* p = nullptr;
+      cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(c, KIE_ERR_CUDA, "cudaGetSymbolAddress(static scratch) failed: %s", cudaGetErrorString(e));
+      }
+      g_static_ptr[c->device] = static_cast<unsigned char*>(p);
+    }
+    base = g_static_ptr[c->device];
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  const kie_config& k = c->cfg;
+  Params P{};
+  P.L = k.n_layers; P.d = k.d_model; P.hq = k.n_heads; P.hk = k.n_kv_heads; P.dh = k.head_dim;
+  P.ff = k.ffn; P.V = k.vocab; P.E = k.n_experts; P.top_k = k.top_k; P.ffe = k.ffn_expert;
+  P.ffs = k.ffn_shared; P.max_ctx = k.max_ctx; P.eps = k.rms_eps;
+  P.qkv_rows = (k.n_heads + 2 * k.n_kv_heads) * k.head_dim;
+  P.slots = c->slots;
+  P.tape = c->tape; P.desc = c->desc;
+  for (int i = 0; i < SK_COUNT; ++i) P.shp[i] = c->shp[i];
+  P.embed = c->embed; P.attn_norm = c->attn_norm; P.mlp_norm = c->mlp_norm;
+  P.final_norm = c->final_norm; P.router = c->router;
+  P.kcache = c->kcache; P.vcache = c->vcache; P.rope = c->rope;
+  P.x = reinterpret_cast<float*>(base + lay.x);
+  P.qkv = reinterpret_cast<float*>(base + lay.qkv);
+  P.o = reinterpret_cast<float*>(base + lay.o);
+  P.h = reinterpret_cast<float*>(base + lay.h);
+  P.apart = reinterpret_cast<float*>(base + lay.apart);
+  P.ctrl = reinterpret_cast<Ctrl*>(base + lay.sync);
+  P.acnt = reinterpret_cast<unsigned*>(base + lay.sync + sizeof(Ctrl));
+  P.cand = reinterpret_cast<Cand*>(base + lay.cand);
+  P.max_chunks = c->max_chunks;
+  P.pos0 = c->pos; P.n_steps = n; P.first_token = c->pending; P.lm_from_step = 0;
+  P.forced = nullptr; P.out_tokens = out_tokens; P.logits_out = nullptr; P.margins_out = nullptr;
+  P.timeout_ns = 1000ull * 1000000ull;
+  P.fault_cta = -1; P.fault_barrier = -1;
+  P.trace = nullptr; P.trace_cap = 0;
+  P.n_stages = c->n_stages; P.stage_bytes = c->stage_bytes; P.vec_floats = c->vec_floats;
+  // the array keeps the previous call's contents: the barrier counter, the
+  // abort flag and the attention arrival counters must start at zero
+  CUDA_TRY(c, cudaMemsetAsync(base + lay.sync, 0, sizeof(Ctrl) + (size_t)k.n_kv_heads * sizeof(unsigned), st));
+  void* args[] = {&P};
+  cudaError_t e = cudaLaunchCooperativeKernel(kernel_entry(), dim3(c->grid), dim3(kThreads), args, (size_t)c->smem, st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(c, KIE_ERR_CUDA, "cooperative launch failed: %s", cudaGetErrorString(e));
+  }
+  c->launches++;
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) {
+    c->poisoned = true;
+    return fail(c, KIE_ERR_CUDA, "decode kernel failed: %s", cudaGetErrorString(e));
+  }
+  Ctrl ctl{};
+  CUDA_TRY(c, cudaMemcpy(&ctl, base + lay.sync, sizeof(Ctrl), cudaMemcpyDeviceToHost));
+  if (ctl.err) {
+    c->poisoned = true;
+    return fail(c, (kie_status)ctl.err, "device %s (cta %d, step %d, where %d); context poisoned",
+                ctl.err == KIE_ERR_TIMEOUT ? "timeout" : "check failed", ctl.err_cta, ctl.err_step, ctl.err_where);
+  }
+  c->pending = ctl.final_token;
+  c->pos += n;
+  return KIE_OK;
+}

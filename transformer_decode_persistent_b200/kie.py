@@ -19,9 +19,9 @@ KIE_OK = 0
 STATUS = {0: "KIE_OK", -1: "KIE_ERR_INVALID_ARG", -2: "KIE_ERR_STATE", -3: "KIE_ERR_CONTEXT_FULL",
           -4: "KIE_ERR_CUDA", -5: "KIE_ERR_TIMEOUT", -6: "KIE_ERR_DEVICE", -7: "KIE_ERR_OOM"}
 
-EXPORTS = ["kie_create", "kie_load_weights", "kie_prefill", "kie_decode", "kie_rewind",
-           "kie_reset", "kie_destroy", "kie_last_error", "kie_position", "kie_pending",
-           "kie_get_info"]
+EXPORTS = ["kie_create", "kie_load_weights", "kie_prefill", "kie_decode", "kie_decode_static",
+           "kie_rewind", "kie_reset", "kie_destroy", "kie_last_error", "kie_position",
+           "kie_pending", "kie_get_info"]
 
 
 class KieError(RuntimeError):
@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
     L.kie_load_weights.argtypes = [VP, P(kie_tensor), I, VP]
     L.kie_prefill.argtypes = [VP, P(ctypes.c_int32), I, VP]
     L.kie_decode.argtypes = [VP, I, VP, P(kie_decode_opts), VP]
+    L.kie_decode_static.argtypes = [VP, I, VP, VP]
     L.kie_rewind.argtypes = [VP, ctypes.c_int32, ctypes.c_int32]
     L.kie_reset.argtypes = [VP]
     L.kie_destroy.argtypes = [VP]
@@ -83,8 +84,8 @@ def lib() -> ctypes.CDLL:
     L.kie_pending.argtypes = [VP]
     L.kie_pending.restype = ctypes.c_int32
     L.kie_get_info.argtypes = [VP, P(kie_info)]
-    for f in ("kie_create", "kie_load_weights", "kie_prefill", "kie_decode", "kie_rewind",
-              "kie_reset", "kie_destroy", "kie_get_info"):
+    for f in ("kie_create", "kie_load_weights", "kie_prefill", "kie_decode", "kie_decode_static",
+              "kie_rewind", "kie_reset", "kie_destroy", "kie_get_info"):
         getattr(L, f).restype = ctypes.c_int
     _lib = L
     return L
@@ -224,6 +225,15 @@ class Engine:
             self._check(self.L.kie_decode(self.h, int(n), ctypes.c_void_p(optr), ctypes.byref(o),
                                           _stream_ptr(stream)))
         return res
+
+    def decode_static(self, n: int, out, stream=None):
+        """kie_decode_static: n greedy tokens into ``out`` (a CUDA int32 tensor),
+        with the kernel's scratch in the library's static device array."""
+        import torch
+        with torch.cuda.device(self.device):
+            self._check(self.L.kie_decode_static(self.h, int(n), ctypes.c_void_p(out.data_ptr()),
+                                                 ctypes.c_void_p(_stream_ptr(stream))))
+        return out
 
     def reset(self):
         self._check(self.L.kie_reset(self.h))
