@@ -131,6 +131,22 @@ def _dist():
     return ws, rank, local
 
 
+def max_over_ranks(values, device="cuda"):
+    """Element-wise maximum over all ranks (the slowest rank's times)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_value(tokens_per_rank: int, world_size: int, elapsed_ms: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * world_size / (elapsed_ms / 1000.0)
+
+
 def cpu_oracle_sample(shape, weights, budget_s: float, max_steps: int):
     """Time the oracle (as it stands) decoding steps of the workload from an
     empty context; returns (tokens/s, steps, seconds, threads)."""
@@ -267,12 +283,9 @@ def main():
     launches = eng.info()["launches"] - l0
     elapsed_ms = t_all0.elapsed_time(t_all1)
     launch_ms = [a.elapsed_time(b) for a, b in ev]
-    if ws > 1:
-        t = torch.tensor([elapsed_ms, max(launch_ms)], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t[0])
+    elapsed_ms = max_over_ranks([elapsed_ms])[0]
     tokens_total = n * args.steps * ws
-    value = tokens_total / (elapsed_ms / 1000.0)
+    value = job_value(n * args.steps, ws, elapsed_ms)
 
     # roofline of the decode kernel (the only kernel in the timed region)
     kvp = info["kv_bytes_per_pos"]
@@ -304,12 +317,8 @@ def main():
         b.record(stream)
         torch.cuda.synchronize()
         wall = time.perf_counter() - w0
-        e_ms = max(a.elapsed_time(b), wall * 1000.0)
-        if ws > 1:
-            t = torch.tensor([e_ms], device="cuda", dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t[0])
-        e2e = {"value": tokens_total / (e_ms / 1000.0), "unit": UNIT,
+        e_ms = max_over_ranks([max(a.elapsed_time(b), wall * 1000.0)])[0]
+        e2e = {"value": job_value(n * args.steps, ws, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(host_prompt.nbytes), "d2h_bytes_per_step": int(n * 4),
                "includes": "reset + prefill of the 256-token prompt from host memory + decode into pinned host memory"}
 

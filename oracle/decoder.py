@@ -204,6 +204,9 @@ class Decoder:
         self.w16 = weights
         self._w64 = {} if cache_f64 else None
         self.kv = fp16_round if kv_fp16 else f64
+        # gap between the k-th and (k+1)-th router probability of every MoE
+        # decision taken by ``step`` (how close each routing was to a tie)
+        self.route_gaps: list[float] = []
 
     def W(self, name: str) -> np.ndarray:
         if self._w64 is None:
@@ -234,6 +237,8 @@ class Decoder:
         s, p = self.s, f"layers.{l}."
         r = softmax(xn @ self.W(p + "router").T)
         chosen = topk_lowest(r, s.top_k)
+        srt = np.sort(r)[::-1]
+        self.route_gaps.append(float(srt[s.top_k - 1] - srt[s.top_k]))
         wsum = sum(r[e] for e in chosen)
         y = swiglu_ffn(xn, self.W(p + "shared.w_gate"), self.W(p + "shared.w_up"),
                        self.W(p + "shared.w_down"))

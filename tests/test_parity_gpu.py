@@ -82,3 +82,77 @@ def test_dense_2b_prefix():
     gl, ol, gt, _ = forced_sequence_case(s, 0, 6, weights=w)
     check_step_logits(gl, ol, "2.2B")
     check_tokens(gt, ol, "2.2B")
+
+
+MOE_SMALL = S.Shape("moe-small", n_layers=3, d_model=256, n_heads=4, n_kv_heads=2, head_dim=64,
+                    ffn=0, vocab=2000, n_experts=8, top_k=2, ffn_expert=128, ffn_shared=256,
+                    prompt_len=20, decode_len=40, max_ctx=60)
+
+
+def test_moe_small_greedy():
+    # routed top-2 of 8 experts + shared expert, GQA 4:2. The oracle records how
+    # close each routing decision came to a tie; decisions the fp32 engine could
+    # take the other way (gap < 1e-4) would make the comparison meaningless.
+    import oracle as O
+    s = MOE_SMALL
+    w = S.make_weights(s, seed=4, cache=False)
+    ref = O.Decoder(s, w)
+    prompt = S.make_prompt(s, 4)
+    ot, ol, om = ref.greedy(prompt, s.decode_len)
+    assert min(ref.route_gaps) > 1e-4, "a routing decision is within 1e-4 of a tie"
+    eng = make_engine(s, w)
+    eng.prefill(prompt)
+    forced = eng.decode(s.decode_len, forced=ot.astype(np.int32), logits=True)
+    check_step_logits(forced["logits"].cpu().numpy(), ol, "moe-small")
+    check_tokens(forced["tokens"], ol, "moe-small")
+    eng.reset()
+    eng.prefill(prompt)
+    check_free_run(eng.decode(s.decode_len)["tokens"], ot, om)
+
+
+def test_moe_full_size_prefix():
+    # the MoE workload at its full size: prompt 128 and 6 forced steps
+    s = S.MOE
+    w = S.make_weights(s, seed=0)
+    gl, ol, gt, _ = forced_sequence_case(s, 0, 6, weights=w)
+    check_step_logits(gl, ol, "moe")
+    check_tokens(gt, ol, "moe")
+
+
+GQA_LONG = S.Shape("gqa-10:8-long", n_layers=3, d_model=512, n_heads=10, n_kv_heads=8,
+                   head_dim=128, ffn=1024, vocab=3000, prompt_len=5000, decode_len=8,
+                   max_ctx=5008)
+
+
+def test_gqa_long_context_multi_round_attention():
+    # ~5000 positions x 8 KV heads: attention units span several CTAs per head
+    # and several 32-position rounds per warp; 10:8 groups are 1 or 2 heads
+    s = GQA_LONG
+    w = S.make_weights(s, seed=5, cache=False)
+    gl, ol, gt, _ = forced_sequence_case(s, 5, s.decode_len, prompt_len=s.prompt_len, weights=w)
+    check_step_logits(gl, ol, "gqa-long")
+    check_tokens(gt, ol, "gqa-long")
+
+
+def test_long_context_full_size_self_consistency():
+    # The long-context workload at full size (32768-token prompt, GQA 20:8, fp16
+    # KV cache of 3.5 GB). The oracle cannot run a 32K-token 2.2B prefix, so the
+    # check is a property: re-forwarding the last prompt tokens in decode mode
+    # (teacher-forced) after rewinding reproduces the same cache and therefore
+    # bit-identical logits and tokens, and repeated runs are deterministic.
+    s = S.LONG_2B
+    w = S.make_weights(s, seed=0)
+    prompt = S.make_prompt(s, 0)
+    eng = make_engine(s, w, max_ctx=s.prompt_len + 32)
+    eng.prefill(prompt)
+    P = len(prompt)
+    a = eng.decode(16, logits=True)
+    k = 8
+    eng.rewind(P - 1 - k, int(prompt[P - 1 - k]))
+    f = eng.decode(k, forced=prompt[P - k:].astype(np.int32))
+    assert eng.position == P - 1 and eng.pending == int(prompt[-1])
+    b = eng.decode(16, logits=True)
+    assert np.array_equal(a["tokens"], b["tokens"])
+    assert np.array_equal(a["logits"].cpu().numpy(), b["logits"].cpu().numpy())
+    lg = a["logits"].cpu().numpy()
+    assert np.isfinite(lg).all() and (np.std(lg, axis=1) > 0.1).all()

@@ -362,7 +362,8 @@ struct Producer {
       const int gi = i / sh.nk, kj = i - gi * sh.nk;
       const int gp = min(sh.g, sd.nrows - gi * sh.g);
       const unsigned bytes = (unsigned)gp * sh.kc * 2u;
-      if (!put(t + i, base + (size_t)gi * sh.g * sh.K * 2 + (size_t)kj * bytes, bytes)) return false;
+      const unsigned char* src = base + (size_t)gi * sh.g * sh.K * 2 + (size_t)kj * bytes;
+      if (!put(t + i, src, bytes)) return false;
     }
     t += ntiles;
     return true;
@@ -752,10 +753,13 @@ struct Consumer {
       __syncwarp();
       if (lane == 0) mbar_arrive(&sc->empty[sV]);
     }
-    // partials -> shared memory (an empty range gives m = -inf, l = 0)
+    // partials -> shared memory, in the slot of this warp's sub-range (not of
+    // the warp: the warp <-> sub-range map depends on the ring position, and
+    // merging in sub-range order keeps results independent of launch history).
+    // An empty range gives m = -inf, l = 0.
 #pragma unroll
     for (int hh = 0; hh < NH; ++hh) {
-      float* pb = wp + (warp * kMaxHeadsPerGroup + hh) * WS;
+      float* pb = wp + (vs * kMaxHeadsPerGroup + hh) * WS;
       if (lane == 0) {
         pb[0] = m[hh];
         pb[1] = ls[hh];
@@ -812,7 +816,7 @@ struct Consumer {
         default: attn_warp<DH, 4>(ap, uo, vs, wj0, wj1, pos, kpos, vpos, qs, wp, sbuf); break;
       }
       cbar();
-      // merge the consumer warps' partials: warp hh merges head hh
+      // merge the sub-ranges' partials in sub-range order: warp hh merges head hh
       if (warp < nh) {
         const int hh = warp;
         float M = -INFINITY;
