@@ -25,7 +25,7 @@
 #include "kie_internal.h"
 
 namespace kie {
-int kernel_smem_bytes(int vec_floats, int n_stages, int stage_bytes);
+int kernel_smem_bytes(int vec_floats, int n_desc, int n_stages, int stage_bytes);
 int kernel_max_stages();
 const void* kernel_entry();
 }  // namespace kie
@@ -45,7 +45,9 @@ struct kie_ctx {
   int grid = 0;
   int n_stages = 0;
   int stage_bytes = 0;
+  int xplane = 0;          // float offset of the input vector's second plane
   int vec_floats = 0;
+  int gbuf_off = 0;
   int smem = 0;
   int max_chunks = 0;
   int hbuf = 0;
@@ -132,18 +134,47 @@ bool is_device_ptr(const void* p) {
 // g >= 4 (the input vector chunk is reused across g rows) with the fewest
 // chunks; GU kinds need an even g so (gate, up) pairs share a tile.
 SegShape choose_shape(int K, bool pairs, int stage_bytes) {
-  SegShape best{K, 0, 0, 0};
-  for (int nk = 1; nk <= 64; ++nk) {
-    if (K % nk) continue;
-    const int kc = K / nk;
-    if (kc % 8) continue;
-    int g = std::min(kMaxRowsPerTile, stage_bytes / (2 * kc));
+  // First choice: the fewest column blocks that give at least 4 rows per
+  // tile. A split into more blocks wins when its chunks divide evenly over the
+  // 32 lanes (kc a multiple of 256 halves, so the kernel's copy-out GEMV
+  // applies) and its tiles keep at least 3/4 of the first choice's bytes.
+  // With no 4-row split, the tallest tile.
+  auto at = [&](int nk) {
+    SegShape sh{K, 0, nk, 0};
+    if (K % nk || (K / nk) % 8) return sh;
+    sh.kc = K / nk;
+    int g = std::min(kMaxRowsPerTile, stage_bytes / (2 * sh.kc));
     if (pairs) g &= ~1;
-    if (g < 1) continue;
-    if (g >= 4) return SegShape{K, g, nk, kc};
-    if (g > best.g) best = SegShape{K, g, nk, kc};
+    sh.g = std::max(g, 0);
+    return sh;
+  };
+  SegShape best{K, 0, 0, 0}, first4{K, 0, 0, 0};
+  for (int nk = 1; nk <= 64; ++nk) {
+    const SegShape sh = at(nk);
+    if (sh.g < 1) continue;
+    if (sh.g >= 4 && first4.g == 0) first4 = sh;
+    if (sh.g > best.g) best = sh;
   }
-  return best;
+  if (!first4.g) return best;
+  if (first4.kc % 256 == 0) return first4;
+  for (int nk = first4.nk + 1; nk <= 64; ++nk) {
+    const SegShape sh = at(nk);
+    if (sh.g >= 4 && sh.kc % 256 == 0 && 4LL * sh.g * sh.kc >= 3LL * first4.g * first4.kc) return sh;
+  }
+  return first4;
+}
+
+// Tile height evened out over the rows one CTA holds (`rows` split over
+// `grid` CTAs in units of 1 or 2 rows): as few tiles as the chosen height
+// allows, all about the same height, so no tile is a sliver.
+SegShape balance_rows(SegShape sh, int rows, int per, bool pairs, int grid) {
+  const int maxu = (rows / per + grid - 1) / grid;
+  const int maxrows = std::max(1, maxu * per);
+  const int ngroups = (maxrows + sh.g - 1) / sh.g;
+  int g = (maxrows + ngroups - 1) / ngroups;
+  if (pairs) g = (g + 1) & ~1;
+  if (g >= 1 && g <= sh.g) sh.g = g;
+  return sh;
 }
 
 // Rows are handed to CTAs in units: (gate, up) pairs for the FFN kinds and
@@ -273,20 +304,26 @@ kie_status kie_create(const kie_config* cfg, int device, kie_ctx** out) {
   c->hbuf = moe ? (k.ffn_shared + k.top_k * k.ffn_expert) : k.ffn;
   // the vector buffer doubles as attention scratch: q of one KV group, the
   // consumer warps' (max, sum, acc) partials and their 32-position score blocks
-  int vf = std::max({d, hq * dh, c->hbuf,
-                     kMaxHeadsPerGroup * dh + kConsumerWarps * kMaxHeadsPerGroup * (dh + 4 + kAttnSub)});
+  // input vectors are stored as two planes (first / second halves of each
+  // 8-float chunk), the second at xplane
+  const int vmax = std::max({d, hq * dh, c->hbuf});
+  c->xplane = ((vmax / 2) + 3) & ~3;
+  int vf = std::max(2 * c->xplane,
+                    kMaxHeadsPerGroup * dh + kConsumerWarps * kMaxHeadsPerGroup * (dh + 4 + kAttnSub));
   vf = (vf + 3) & ~3;
+  c->gbuf_off = vf;           // then d fp16 norm-gain values
+  vf += ((d / 2) + 3) & ~3;
   c->vec_floats = vf;
   // kRingStages ring stages (two per consumer warp) of the largest size that
   // fits, in 1 KiB steps, at most 16 KiB
-  const int fixed = kernel_smem_bytes(vf, 0, 0);
+  const int fixed = kernel_smem_bytes(vf, 4 * k.n_layers + 1, 0, 0);
   const int optin = (int)prop.sharedMemPerBlockOptin;
   const int ns = kernel_max_stages();
   int sb = std::min(kMaxStageBytes, ((optin - fixed) / ns) & ~1023);
   if (sb < 4096) return bail(fail(c, KIE_ERR_INVALID_ARG, "shape needs too much shared memory"));
   c->n_stages = ns;
   c->stage_bytes = sb;
-  c->smem = kernel_smem_bytes(vf, ns, sb);
+  c->smem = kernel_smem_bytes(vf, 4 * k.n_layers + 1, ns, sb);
   if (cudaFuncSetAttribute(kernel_entry(), cudaFuncAttributeMaxDynamicSharedMemorySize, c->smem) !=
       cudaSuccess)
     return bail(fail(c, KIE_ERR_CUDA, "cudaFuncSetAttribute(smem=%d) failed: %s", c->smem,
@@ -297,6 +334,9 @@ kie_status kie_create(const kie_config* cfg, int device, kie_ctx** out) {
       per_sm < 1)
     return bail(fail(c, KIE_ERR_CUDA, "kernel does not fit on an SM (smem %d)", c->smem));
   c->grid = c->sms;  // one CTA per SM; the ring takes the SM's shared memory
+  if ((d + c->grid - 1) / c->grid > kMaxOwnRows)
+    return bail(fail(c, KIE_ERR_INVALID_ARG, "d_model %d over %d CTAs exceeds %d residual rows per CTA", d,
+                     c->grid, kMaxOwnRows));
   c->slots = slots_per_layer(moe ? k.n_experts : 0);
 
   // attention units cover >= 256 positions and >= T*hk/grid positions each
@@ -497,17 +537,20 @@ kie_status kie_load_weights(kie_ctx* c, const kie_tensor* tensors, int n, void* 
 
   // segment shapes
   const int ffs = k.ffn_shared, ffe = k.ffn_expert;
-  c->shp[SK_QKV] = choose_shape(d, false, c->stage_bytes);
-  c->shp[SK_O] = choose_shape(hq * dh, false, c->stage_bytes);
-  c->shp[SK_LM] = choose_shape(d, false, c->stage_bytes);
-  if (!moe) {
-    c->shp[SK_GU] = choose_shape(d, true, c->stage_bytes);
-    c->shp[SK_DOWN] = choose_shape(k.ffn, false, c->stage_bytes);
-  } else {
-    c->shp[SK_SGU] = choose_shape(d, true, c->stage_bytes);
-    c->shp[SK_EGU] = choose_shape(d, true, c->stage_bytes);
-    c->shp[SK_SDOWN] = choose_shape(ffs, false, c->stage_bytes);
-    c->shp[SK_EDOWN] = choose_shape(ffe, false, c->stage_bytes);
+  {
+    const int G = c->grid, sb = c->stage_bytes;
+    c->shp[SK_QKV] = balance_rows(choose_shape(d, false, sb), (hq + 2 * hk) * dh, 2, false, G);
+    c->shp[SK_O] = balance_rows(choose_shape(hq * dh, false, sb), d, 1, false, G);
+    c->shp[SK_LM] = balance_rows(choose_shape(d, false, sb), k.vocab, 1, false, G);
+    if (!moe) {
+      c->shp[SK_GU] = balance_rows(choose_shape(d, true, sb), 2 * k.ffn, 2, true, G);
+      c->shp[SK_DOWN] = balance_rows(choose_shape(k.ffn, false, sb), d, 1, false, G);
+    } else {
+      c->shp[SK_SGU] = balance_rows(choose_shape(d, true, sb), 2 * ffs, 2, true, G);
+      c->shp[SK_EGU] = balance_rows(choose_shape(d, true, sb), 2 * ffe, 2, true, G);
+      c->shp[SK_SDOWN] = balance_rows(choose_shape(ffs, false, sb), d, 1, false, G);
+      c->shp[SK_EDOWN] = balance_rows(choose_shape(ffe, false, sb), d, 1, false, G);
+    }
   }
 
   // row assignment
@@ -516,16 +559,18 @@ kie_status kie_load_weights(kie_ctx* c, const kie_tensor* tensors, int n, void* 
   for (int l = 0; l < L; ++l) {
     const int rot = (int)(((long long)l * 53) % G);
     pl.assign(l, 0, SK_QKV, (hq + 2 * hk) * dh, rot);
-    pl.assign(l, 1, SK_O, d, (rot + 17) % G);
+    // the output and down projections own the same residual rows in every
+    // layer (no rotation): each CTA keeps its rows in shared memory
+    pl.assign(l, 1, SK_O, d, 0);
     if (!moe) {
       pl.assign(l, 2, SK_GU, 2 * k.ffn, (rot + 31) % G);
-      pl.assign(l, 3, SK_DOWN, d, (rot + 71) % G);
+      pl.assign(l, 3, SK_DOWN, d, 0);
     } else {
       pl.assign(l, 2, SK_SGU, 2 * ffs, (rot + 31) % G);
-      pl.assign(l, 3, SK_SDOWN, d, (rot + 71) % G);
+      pl.assign(l, 3, SK_SDOWN, d, 0);
       for (int e = 0; e < k.n_experts; ++e) {
         pl.assign(l, 4 + e, SK_EGU, 2 * ffe, (rot + 97 + 7 * e) % G);
-        pl.assign(l, 4 + k.n_experts + e, SK_EDOWN, d, (rot + 71) % G);  // same rows as SDOWN
+        pl.assign(l, 4 + k.n_experts + e, SK_EDOWN, d, 0);
       }
     }
   }
@@ -765,6 +810,8 @@ kie_status launch(kie_ctx* c, const Run& r, cudaStream_t st) {
   P.fault_cta = r.fault_cta; P.fault_barrier = r.fault_barrier;
   P.trace = reinterpret_cast<unsigned long long*>(r.trace); P.trace_cap = r.trace_cap;
   P.n_stages = c->n_stages; P.stage_bytes = c->stage_bytes; P.vec_floats = c->vec_floats;
+  P.xplane = c->xplane;
+  P.gbuf_off = c->gbuf_off;
 
   CUDA_TRY(c, cudaMemsetAsync(c->syncblk, 0, c->syncblk_bytes, st));
   void* args[] = {&P};
@@ -1023,6 +1070,8 @@ extern "C" kie_status kie_decode_static(kie_ctx* c, int n, int32_t* out_tokens, 
   P.fault_cta = -1; P.fault_barrier = -1;
   P.trace = nullptr; P.trace_cap = 0;
   P.n_stages = c->n_stages; P.stage_bytes = c->stage_bytes; P.vec_floats = c->vec_floats;
+  P.xplane = c->xplane;
+  P.gbuf_off = c->gbuf_off;
   // the array keeps the previous call's contents: the barrier counter, the
   // abort flag and the attention arrival counters must start at zero
   CUDA_TRY(c, cudaMemsetAsync(base + lay.sync, 0, sizeof(Ctrl) + (size_t)k.n_kv_heads * sizeof(unsigned), st));

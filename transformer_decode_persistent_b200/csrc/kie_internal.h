@@ -22,6 +22,7 @@ constexpr int kMaxHeadsPerGroup = 4;                   // query heads per KV hea
 constexpr int kMaxTopK = 4;                            // routed experts per token
 constexpr int kAttnSub = 32;                           // positions per attention sub-block
 constexpr int kMaxExperts = 64;
+constexpr int kMaxOwnRows = 64;                        // residual rows a CTA keeps in shared memory
 
 // ---- weight tape ------------------------------------------------------------
 // The tape is one device buffer. CTA c owns a contiguous region holding, in
@@ -122,7 +123,9 @@ struct Params {
   int trace_cap;
   int n_stages;     // multiple of kConsumerWarps: stage s belongs to warp s % kConsumerWarps
   int stage_bytes;
-  int vec_floats;
+  int vec_floats;   // shared vector buffer, including the norm-gain buffer at gbuf_off
+  int gbuf_off;     // float offset of the fp16 norm-gain buffer inside the vector buffer
+  int xplane;       // float offset of the second-half plane of the input vector (see Consumer::xv)
 };
 
 }  // namespace kie

@@ -55,17 +55,38 @@ struct SmemCtl {
   float red[64];
   Cand wcand[kConsumerWarps];
   unsigned bcast;
+  // this CTA's rows of the residual stream: the output projection and the
+  // FFN down projection own the same rows in every layer
+  float xown[kMaxOwnRows];
 };
 
 // Shared-memory layout, identical on host and device.
 __host__ __device__ inline int smem_ctl_bytes() { return (int)((sizeof(SmemCtl) + 127) & ~127); }
-__host__ __device__ inline int smem_ring_offset(int vec_floats) {
-  int b = smem_ctl_bytes() + kPartFloats * 4 + vec_floats * 4;
+// control block | partial sums | vector buffer | descriptor cache | ring
+__host__ __device__ inline int smem_desc_offset(int vec_floats) {
+  return (smem_ctl_bytes() + kPartFloats * 4 + vec_floats * 4 + 15) & ~15;
+}
+__host__ __device__ inline int smem_ring_offset(int vec_floats, int n_desc) {
+  const int b = smem_desc_offset(vec_floats) + n_desc * (int)sizeof(SegDesc);
   return (b + 1023) & ~1023;
 }
-__host__ __device__ inline int smem_total(int vec_floats, int n_stages, int stage_bytes) {
-  return smem_ring_offset(vec_floats) + n_stages * stage_bytes;
+__host__ __device__ inline int smem_total(int vec_floats, int n_desc, int n_stages, int stage_bytes) {
+  return smem_ring_offset(vec_floats, n_desc) + n_stages * stage_bytes;
 }
+
+// This CTA's descriptors of the per-layer segments q/k/v, o, gate/up and down
+// (slots 0..3) and of the LM head, copied to shared memory at launch so that a
+// phase does not start with a global load. Routed experts' descriptors stay in
+// global memory.
+struct DescCache {
+  const SegDesc* sm;  // [4 L + 1]
+  const SegDesc* g;   // this CTA's global descriptors [L * slots + 1]
+  int L, slots;
+  __device__ __forceinline__ const SegDesc& at(int l, int slot) const {
+    if (l == L) return sm[4 * L];
+    return slot < 4 ? sm[4 * l + slot] : g[(size_t)l * slots + slot];
+  }
+};
 
 // ---------------------------------------------------------------- primitives
 
@@ -337,8 +358,10 @@ struct Producer {
   unsigned mine = 0;  // tiles issued by this lane
   int step = 0;
 
-  __device__ Producer(const Params& p, SmemCtl* s, unsigned char* r, int ln)
-      : P(p), sc(s), ring(r), lane(ln) {
+  const DescCache dc;
+
+  __device__ Producer(const Params& p, SmemCtl* s, unsigned char* r, int ln, const DescCache& d)
+      : P(p), sc(s), ring(r), lane(ln), dc(d) {
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
   }
 
@@ -413,18 +436,16 @@ struct Producer {
 
   __device__ void run() {
     const int c = blockIdx.x;
-    const SegDesc* D = P.desc + (size_t)c * (P.L * P.slots + 1);
     bool ok = true;
     unsigned route_round = 0;
     for (step = 0; ok && step < P.n_steps; ++step) {
       for (int l = 0; ok && l < P.L; ++l) {
-        const SegDesc* Dl = D + (size_t)l * P.slots;
-        ok = issue(Dl[0], P.shp[SK_QKV]) && issue_attn(l, P.pos0 + step) && issue(Dl[1], P.shp[SK_O]);
+        ok = issue(dc.at(l, 0), P.shp[SK_QKV]) && issue_attn(l, P.pos0 + step) && issue(dc.at(l, 1), P.shp[SK_O]);
         if (!ok) break;
         if (P.E == 0) {
-          ok = issue(Dl[2], P.shp[SK_GU]) && issue(Dl[3], P.shp[SK_DOWN]);
+          ok = issue(dc.at(l, 2), P.shp[SK_GU]) && issue(dc.at(l, 3), P.shp[SK_DOWN]);
         } else {
-          ok = issue(Dl[2], P.shp[SK_SGU]);
+          ok = issue(dc.at(l, 2), P.shp[SK_SGU]);
           if (!ok) break;
           // the routed experts are known only once the consumers have run the router
           ok = wait_route(route_round);
@@ -432,12 +453,12 @@ struct Producer {
           int e[kMaxTopK];
           for (int k = 0; k < P.top_k; ++k) e[k] = sc->route_e[route_round % kRouteRing][k];
           ++route_round;
-          for (int k = 0; ok && k < P.top_k; ++k) ok = issue(Dl[4 + e[k]], P.shp[SK_EGU]);
-          ok = ok && issue(Dl[3], P.shp[SK_SDOWN]);
-          for (int k = 0; ok && k < P.top_k; ++k) ok = issue(Dl[4 + P.E + e[k]], P.shp[SK_EDOWN]);
+          for (int k = 0; ok && k < P.top_k; ++k) ok = issue(dc.at(l, 4 + e[k]), P.shp[SK_EGU]);
+          ok = ok && issue(dc.at(l, 3), P.shp[SK_SDOWN]);
+          for (int k = 0; ok && k < P.top_k; ++k) ok = issue(dc.at(l, 4 + P.E + e[k]), P.shp[SK_EDOWN]);
         }
       }
-      if (ok && step >= P.lm_from_step) ok = issue(D[(size_t)P.L * P.slots], P.shp[SK_LM]);
+      if (ok && step >= P.lm_from_step) ok = issue(dc.at(P.L, 0), P.shp[SK_LM]);
     }
     // let this lane's last copy land before the CTA may exit
     if (mine > 0) {
@@ -453,26 +474,61 @@ struct Producer {
 // ---------------------------------------------------------------- consumer
 
 // One tile: G rows x nch 16-byte chunks, row-major in the stage at shared
-// address w_s; the fp32 input slice at x_s. Lane l takes chunks l, l+32, ...;
+// address w_s; the fp32 input slice in the split layout of the vector buffer
+// (first halves of the 8-float chunks at x_s, second halves xpb bytes on, so a
+// warp's 16-byte loads are contiguous). Lane l takes chunks l, l+32, ...;
 // the input chunk is read once and reused for all G rows. Writes the G row
 // partial sums to part[pidx0 + r * pstride].
 template <int G>
-__device__ __forceinline__ void tile_gemv(uint32_t w_s, uint32_t x_s, int nch, int lane, float* part,
-                                          int pidx0, int pstride) {
+__device__ __forceinline__ void tile_gemv(uint32_t w_s, uint32_t x_s, uint32_t xpb, int nch, int lane, float* part,
+                                          int pidx0, int pstride, uint64_t* empty) {
   float acc[G];
 #pragma unroll
   for (int r = 0; r < G; ++r) acc[r] = 0.f;
 #pragma unroll 2
   for (int c = lane; c < nch; c += 32) {
-    const float4 a = lds_f4(x_s + c * 32);
-    const float4 b = lds_f4(x_s + c * 32 + 16);
+    const float4 a = lds_f4(x_s + c * 16);
+    const float4 b = lds_f4(x_s + xpb + c * 16);
 #pragma unroll
     for (int r = 0; r < G; ++r) acc[r] = dot8(lds_u4(w_s + (uint32_t)(r * nch + c) * 16u), a, b, acc[r]);
   }
   __syncwarp();
+  if (lane == 0) mbar_arrive(empty);  // stage free for the next copy
 #pragma unroll
   for (int r = 0; r < G; ++r) {
     const float v = warp_sum(acc[r]);
+    if (lane == r) part[pidx0 + r * pstride] = v;
+  }
+}
+
+// Same product for full tiles of G rows and 32*CPL chunks: the lane's whole
+// share of the tile is first copied to registers, the stage is released at
+// once (so its next bulk copy starts about a GEMV earlier), then the math runs
+// from registers.
+template <int G, int CPL>
+__device__ __forceinline__ void tile_gemv_copyout(uint32_t w_s, uint32_t x_s, uint32_t xpb, int lane, float* part,
+                                                  int pidx0, int pstride, uint64_t* empty) {
+  constexpr int nch = CPL * 32;
+  uint4 wr[G][CPL];
+#pragma unroll
+  for (int k = 0; k < CPL; ++k)
+#pragma unroll
+    for (int r = 0; r < G; ++r) wr[r][k] = lds_u4(w_s + (uint32_t)(r * nch + lane + 32 * k) * 16u);
+  __syncwarp();
+  if (lane == 0) mbar_arrive(empty);
+  float acc[G][2];
+#pragma unroll
+  for (int r = 0; r < G; ++r) acc[r][0] = acc[r][1] = 0.f;
+#pragma unroll
+  for (int k = 0; k < CPL; ++k) {
+    const uint32_t xa = x_s + (uint32_t)(lane + 32 * k) * 16u;
+    const float4 a = lds_f4(xa), b = lds_f4(xa + xpb);
+#pragma unroll
+    for (int r = 0; r < G; ++r) acc[r][k & 1] = dot8(wr[r][k], a, b, acc[r][k & 1]);
+  }
+#pragma unroll
+  for (int r = 0; r < G; ++r) {
+    const float v = warp_sum(acc[r][0] + acc[r][1]);
     if (lane == r) part[pidx0 + r * pstride] = v;
   }
 }
@@ -489,9 +545,11 @@ struct Consumer {
   int step = 0;
   unsigned route_round = 0;
 
-  __device__ Consumer(const Params& p, SmemCtl* s, float* pa, float* v, unsigned char* r)
+  const DescCache dc;
+
+  __device__ Consumer(const Params& p, SmemCtl* s, float* pa, float* v, unsigned char* r, const DescCache& d)
       : P(p), sc(s), part(pa), vec(v), ring(r), tid(threadIdx.x), warp(threadIdx.x >> 5),
-        lane(threadIdx.x & 31) {}
+        lane(threadIdx.x & 31), dc(d) {}
 
   __device__ float block_sum(float v) {
     v = warp_sum(v);
@@ -504,21 +562,35 @@ struct Consumer {
     return t;
   }
 
-  // vec[0..n) = src (fp32, L2-resident scratch)
+  // The vector buffer holds an input vector split by halves of its 8-float
+  // chunks: element i of chunk c (i < 4) at vec[4c + i], element 4 + i at
+  // vec[xplane + 4c + i]. xv(i) is where the 4 elements from i (i % 4 == 0) go.
+  __device__ __forceinline__ float* xv(int i) const {
+    return vec + ((i & 4) ? P.xplane : 0) + ((i >> 3) << 2);
+  }
+
+  // vec = src (fp32, L2-resident scratch), n a multiple of 8
   __device__ void load_vec(const float* src, int n) {
     for (int i = tid * 4; i < n; i += kConsumerThreads * 4)
-      *reinterpret_cast<float4*>(vec + i) = *reinterpret_cast<const float4*>(src + i);
+      *reinterpret_cast<float4*>(xv(i)) = *reinterpret_cast<const float4*>(src + i);
     cbar();
   }
 
+  // Start copying the next RMSNorm gain into the shared gain buffer
+  // (cp.async, no registers held); load_norm waits for it. Issued right after
+  // the previous load_norm, so the copy overlaps a whole phase.
+  __device__ void prefetch_gain(const __half* g) {
+    const uint32_t gb = su32(vec + P.gbuf_off);
+    for (int i = tid * 8; i < P.d; i += kConsumerThreads * 8)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(gb + i * 2), "l"(g + i) : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+
   // vec = RMSNorm(src) * gain, src either fp32 (residual) or an fp16 embedding
-  // row. The (read-only) gain is prefetched into L1 alongside the source loads,
-  // so the scaling pass after the block reduction does not pay a second L2
-  // round trip.
-  __device__ void load_norm(const float* srcf, const __half* srch, const __half* gain, int n) {
+  // row; the gain was prefetched into the gain buffer by prefetch_gain.
+  __device__ void load_norm(const float* srcf, const __half* srch, int n) {
     float ss = 0.f;
     for (int i = tid * 4; i < n; i += kConsumerThreads * 4) {
-      asm volatile("prefetch.global.L1 [%0];" ::"l"(gain + i));
       float4 v;
       if (srcf) {
         v = *reinterpret_cast<const float4*>(srcf + i);
@@ -527,19 +599,22 @@ struct Consumer {
         const float2 lo = h2f2(raw.x), hi = h2f2(raw.y);
         v = make_float4(lo.x, lo.y, hi.x, hi.y);
       }
-      *reinterpret_cast<float4*>(vec + i) = v;
+      *reinterpret_cast<float4*>(xv(i)) = v;
       ss = fmaf(v.x, v.x, ss);
       ss = fmaf(v.y, v.y, ss);
       ss = fmaf(v.z, v.z, ss);
       ss = fmaf(v.w, v.w, ss);
     }
-    const float tot = block_sum(ss);
+    asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's gain copies
+    const float tot = block_sum(ss);                   // (its barrier publishes all of them)
     const float inv = 1.0f / sqrtf(tot / (float)n + P.eps);
+    const __half* gb = reinterpret_cast<const __half*>(vec + P.gbuf_off);
     for (int i = tid * 4; i < n; i += kConsumerThreads * 4) {
-      const uint2 g = __ldg(reinterpret_cast<const uint2*>(gain + i));
+      const uint2 g = *reinterpret_cast<const uint2*>(gb + i);
       const float2 g0 = h2f2(g.x), g1 = h2f2(g.y);
-      const float4 v = *reinterpret_cast<const float4*>(vec + i);
-      *reinterpret_cast<float4*>(vec + i) = make_float4(v.x * inv * g0.x, v.y * inv * g0.y, v.z * inv * g1.x, v.w * inv * g1.y);
+      float4* xp = reinterpret_cast<float4*>(xv(i));
+      const float4 v = *xp;
+      *xp = make_float4(v.x * inv * g0.x, v.y * inv * g0.y, v.z * inv * g1.x, v.w * inv * g1.y);
     }
     cbar();
   }
@@ -556,28 +631,60 @@ struct Consumer {
     // used by one warp, in order: its parity waits can never see a phase two
     // rounds old.
     const int first = (int)((warp + kConsumerWarps - (int)(tbase % kConsumerWarps)) % kConsumerWarps);
+    // stage, parity and (row group, column block) of this warp's tiles,
+    // advanced without divisions: each step is kConsumerWarps tiles on
+    const unsigned t0 = tbase + (unsigned)first;
+    int s = (int)(t0 % (unsigned)ns);
+    unsigned par = (t0 / (unsigned)ns) & 1u;
+    int gi = first / sh.nk, kj = first - gi * sh.nk;
+    const int dg = kConsumerWarps / sh.nk, dk = kConsumerWarps - dg * sh.nk;
     for (int i = first; i < ntiles; i += kConsumerWarps) {
       if (sc->abort) break;
-      const unsigned t = tbase + i;
-      const int s = (int)(t % ns);
-      if (!wait_bar(P, sc, &sc->full[s], (t / ns) & 1u, 2, step)) break;
-      const int gi = i / sh.nk, kj = i - gi * sh.nk;
+      if (!wait_bar(P, sc, &sc->full[s], par, 2, step)) break;
       const int gp = min(sh.g, sd.nrows - gi * sh.g);
       const uint32_t w = su32(ring) + (uint32_t)(s * P.stage_bytes);
-      const uint32_t xv = su32(vseg) + (uint32_t)(kj * sh.kc) * 4u;
+      const uint32_t xs = su32(vseg) + (uint32_t)(kj * sh.kc) * 2u;
+      const uint32_t xpb = (uint32_t)P.xplane * 4u;
       const int p0 = pbase + gi * sh.g * pstride + kjbase + kj;
-      // the stage is released inside tile_gemv's reduction (after __syncwarp)
-      switch (gp) {
-        case 1: tile_gemv<1>(w, xv, nch, lane, part, p0, pstride); break;
-        case 2: tile_gemv<2>(w, xv, nch, lane, part, p0, pstride); break;
-        case 3: tile_gemv<3>(w, xv, nch, lane, part, p0, pstride); break;
-        case 4: tile_gemv<4>(w, xv, nch, lane, part, p0, pstride); break;
-        case 5: tile_gemv<5>(w, xv, nch, lane, part, p0, pstride); break;
-        case 6: tile_gemv<6>(w, xv, nch, lane, part, p0, pstride); break;
-        case 7: tile_gemv<7>(w, xv, nch, lane, part, p0, pstride); break;
-        default: tile_gemv<8>(w, xv, nch, lane, part, p0, pstride); break;
+      uint64_t* em = &sc->empty[s];
+      bool done = false;
+      if (gp == sh.g && (nch & 31) == 0) {
+        done = true;
+        switch (gp * 16 + (nch >> 5)) {
+          case 8 * 16 + 1: tile_gemv_copyout<8, 1>(w, xs, xpb, lane, part, p0, pstride, em); break;
+          case 8 * 16 + 3: tile_gemv_copyout<8, 3>(w, xs, xpb, lane, part, p0, pstride, em); break;
+          case 6 * 16 + 3: tile_gemv_copyout<6, 3>(w, xs, xpb, lane, part, p0, pstride, em); break;
+          case 4 * 16 + 5: tile_gemv_copyout<4, 5>(w, xs, xpb, lane, part, p0, pstride, em); break;
+          case 5 * 16 + 5: tile_gemv_copyout<5, 5>(w, xs, xpb, lane, part, p0, pstride, em); break;
+          case 4 * 16 + 6: tile_gemv_copyout<4, 6>(w, xs, xpb, lane, part, p0, pstride, em); break;
+          case 6 * 16 + 4: tile_gemv_copyout<6, 4>(w, xs, xpb, lane, part, p0, pstride, em); break;
+          case 7 * 16 + 4: tile_gemv_copyout<7, 4>(w, xs, xpb, lane, part, p0, pstride, em); break;
+          default: done = false;
+        }
       }
-      if (lane == 0) mbar_arrive(&sc->empty[s]);
+      if (!done) {
+        switch (gp) {
+          case 1: tile_gemv<1>(w, xs, xpb, nch, lane, part, p0, pstride, em); break;
+          case 2: tile_gemv<2>(w, xs, xpb, nch, lane, part, p0, pstride, em); break;
+          case 3: tile_gemv<3>(w, xs, xpb, nch, lane, part, p0, pstride, em); break;
+          case 4: tile_gemv<4>(w, xs, xpb, nch, lane, part, p0, pstride, em); break;
+          case 5: tile_gemv<5>(w, xs, xpb, nch, lane, part, p0, pstride, em); break;
+          case 6: tile_gemv<6>(w, xs, xpb, nch, lane, part, p0, pstride, em); break;
+          case 7: tile_gemv<7>(w, xs, xpb, nch, lane, part, p0, pstride, em); break;
+          default: tile_gemv<8>(w, xs, xpb, nch, lane, part, p0, pstride, em); break;
+        }
+      }
+      s += kConsumerWarps;
+      if (s >= ns) {
+        s -= ns;
+        par ^= 1u;
+      }
+      kj += dk;
+      gi += dg;
+      if (kj >= sh.nk) {
+        kj -= sh.nk;
+        ++gi;
+      }
     }
     tbase += ntiles;
   }
@@ -951,12 +1058,15 @@ struct Consumer {
     asm volatile("fence.proxy.async.global;" ::: "memory");
   }
 
-  // residual epilogue: x[row] = xprev[row] + sum of partials
+  // residual epilogue: x[row] = xprev[row] + sum of partials. xprev is this
+  // CTA's own copy of its rows (or the embedding row in the first layer).
   __device__ void epi_residual(const SegDesc& sd, int stride, const __half* xprev_h) {
     for (int r = tid; r < sd.nrows; r += kConsumerThreads) {
       const int row = sd.row0 + r;
-      const float xp = xprev_h ? __half2float(xprev_h[row]) : P.x[row];
-      P.x[row] = xp + row_sum(r, stride);
+      const float xp = xprev_h ? __half2float(xprev_h[row]) : sc->xown[r];
+      const float v = xp + row_sum(r, stride);
+      sc->xown[r] = v;
+      P.x[row] = v;
     }
   }
 
@@ -981,8 +1091,8 @@ struct Consumer {
       float a = 0.f;
       for (int c = lane; c < P.d / 8; c += 32) {
         const uint4 wv = *reinterpret_cast<const uint4*>(row + c * 8);
-        a = dot8(wv, *reinterpret_cast<const float4*>(vec + c * 8),
-                 *reinterpret_cast<const float4*>(vec + c * 8 + 4), a);
+        a = dot8(wv, *reinterpret_cast<const float4*>(xv(c * 8)),
+                 *reinterpret_cast<const float4*>(xv(c * 8 + 4)), a);
       }
       a = warp_sum(a);
       if (lane == 0) part[e] = a;
@@ -1017,145 +1127,132 @@ struct Consumer {
     ++route_round;
   }
 
-  __device__ bool layer(int l, int tok, int pos, const SegDesc* D) {
-    const SegDesc* Dl = D + (size_t)l * P.slots;
-    const __half* erow = P.embed + (size_t)tok * P.d;
-    // ---- q, k, v projections of RMSNorm(x)
-    if (l == 0) load_norm(nullptr, erow, P.attn_norm, P.d);
-    else load_norm(P.x, nullptr, P.attn_norm + (size_t)l * P.d, P.d);
-    const SegShape& sq = P.shp[SK_QKV];
-    run_segment(Dl[0], sq, vec, 0, sq.nk, 0);
-    cbar();
-    epi_qkv(Dl[0], sq.nk, l, pos);
-    if (!grid_sync()) return false;
-    // ---- RoPE, KV append, attention
-    attention_dispatch(l, pos);
-    if (!grid_sync()) return false;
-    // ---- output projection + residual
-    load_vec(P.o, P.hq * P.dh);
-    const SegShape& so = P.shp[SK_O];
-    run_segment(Dl[1], so, vec, 0, so.nk, 0);
-    cbar();
-    epi_residual(Dl[1], so.nk, l == 0 ? erow : nullptr);
-    if (!grid_sync()) return false;
-    // ---- FFN
-    load_norm(P.x, nullptr, P.mlp_norm + (size_t)l * P.d, P.d);
-    if (P.E == 0) {
-      const SegShape& sg = P.shp[SK_GU];
-      run_segment(Dl[2], sg, vec, 0, sg.nk, 0);
-      cbar();
-      epi_swiglu(Dl[2], 0, sg.nk, 0, 1.0f);
-      if (!grid_sync()) return false;
-      load_vec(P.h, P.ff);
-      const SegShape& sd = P.shp[SK_DOWN];
-      run_segment(Dl[3], sd, vec, 0, sd.nk, 0);
-      cbar();
-      epi_residual(Dl[3], sd.nk, nullptr);
-      if (!grid_sync()) return false;
-    } else {
-      const int* re = sc->route_e[route_round % kRouteRing];
-      route(l);
-      int e[kMaxTopK];
-      float w[kMaxTopK];
-      for (int k = 0; k < P.top_k; ++k) {
-        e[k] = re[k];
-        w[k] = sc->route_w[k];
-      }
-      const SegShape& ss = P.shp[SK_SGU];
-      const SegShape& se = P.shp[SK_EGU];
-      const SegDesc& dsh = Dl[2];
-      run_segment(dsh, ss, vec, 0, ss.nk, 0);
-      int pb[kMaxTopK];
-      int pnext = dsh.nrows * ss.nk;
-      for (int k = 0; k < P.top_k; ++k) {
-        pb[k] = pnext;
-        const SegDesc& de = Dl[4 + e[k]];
-        run_segment(de, se, vec, pb[k], se.nk, 0);
-        pnext += de.nrows * se.nk;
-      }
-      cbar();
-      epi_swiglu(dsh, 0, ss.nk, 0, 1.0f);
-      for (int k = 0; k < P.top_k; ++k) epi_swiglu(Dl[4 + e[k]], pb[k], se.nk, P.ffs + k * P.ffe, w[k]);
-      if (!grid_sync()) return false;
-      load_vec(P.h, P.ffs + P.top_k * P.ffe);
-      const SegShape& sds = P.shp[SK_SDOWN];
-      const SegShape& sde = P.shp[SK_EDOWN];
-      const int stride = sds.nk + P.top_k * sde.nk;
-      run_segment(Dl[3], sds, vec, 0, stride, 0);
-      for (int k = 0; k < P.top_k; ++k)
-        run_segment(Dl[4 + P.E + e[k]], sde, vec + P.ffs + k * P.ffe, 0, stride, sds.nk + k * sde.nk);
-      cbar();
-      epi_residual(Dl[3], stride, nullptr);
-      if (!grid_sync()) return false;
-    }
-    return true;
-  }
+  // The per-token step as a sequence of phases separated by grid barriers:
+  // per layer q/k/v, attention, output projection, FFN up (gate/up or routed
+  // experts), FFN down; then the LM head when the step samples. Every phase
+  // reads its input vector, runs its tiles through the one run_segment call
+  // site (one inlined copy of the GEMV code keeps the instruction cache warm),
+  // then runs its epilogue.
+  enum PhaseKind { PH_QKV = 0, PH_ATTN = 1, PH_O = 2, PH_UP = 3, PH_DOWN = 4, PH_LM = 5 };
 
   __device__ void run() {
     const int c = blockIdx.x;
-    const SegDesc* D = P.desc + (size_t)c * (P.L * P.slots + 1);
     int tok = P.first_token;
+    prefetch_gain(P.attn_norm);
     for (step = 0; step < P.n_steps; ++step) {
       const int pos = P.pos0 + step;
       if (tok < 0 || tok >= P.V) {
         if (tid == 0) record_error(P, kErrDevice, 5, step);
         return;
       }
-      for (int l = 0; l < P.L; ++l)
-        if (!layer(l, tok, pos, D)) return;
-      int next;
-      if (step >= P.lm_from_step) {
-        // ---- final norm, LM head, greedy argmax
-        load_norm(P.x, nullptr, P.final_norm, P.d);
-        const SegDesc& dl = D[(size_t)P.L * P.slots];
-        const SegShape& sl = P.shp[SK_LM];
-        run_segment(dl, sl, vec, 0, sl.nk, 0);
-        cbar();
-        float v1 = -INFINITY, v2 = -INFINITY;
-        int i1 = INT_MAX;
-        for (int r = tid; r < dl.nrows; r += kConsumerThreads) {
-          const float y = row_sum(r, sl.nk);
-          const int row = dl.row0 + r;
-          if (P.logits_out) P.logits_out[(size_t)step * P.V + row] = y;
-          cand_merge(v1, i1, v2, y, row, -INFINITY);
+      const bool lm = step >= P.lm_from_step;
+      const __half* erow = P.embed + (size_t)tok * P.d;
+      const int nph = P.L * 5 + (lm ? 1 : 0);
+      int re[kMaxTopK];
+      float rw[kMaxTopK];
+      int rpb[kMaxTopK];
+      for (int ph = 0; ph < nph; ++ph) {
+        const int l = ph / 5;
+        const int kind = (l == P.L) ? PH_LM : ph - l * 5;
+        // ---- 1. input vector
+        switch (kind) {
+          case PH_QKV:
+            if (l == 0) load_norm(nullptr, erow, P.d);
+            else load_norm(P.x, nullptr, P.d);
+            prefetch_gain(P.mlp_norm + (size_t)l * P.d);
+            break;
+          case PH_O:
+            load_vec(P.o, P.hq * P.dh);
+            break;
+          case PH_UP:
+            load_norm(P.x, nullptr, P.d);
+            if (l + 1 < P.L) prefetch_gain(P.attn_norm + (size_t)(l + 1) * P.d);
+            else prefetch_gain(lm ? P.final_norm : P.attn_norm);
+            if (P.E) {
+              const int* pick = sc->route_e[route_round % kRouteRing];
+              route(l);
+              for (int k = 0; k < P.top_k; ++k) {
+                re[k] = pick[k];
+                rw[k] = sc->route_w[k];
+              }
+            }
+            break;
+          case PH_DOWN:
+            load_vec(P.h, P.E ? P.ffs + P.top_k * P.ffe : P.ff);
+            break;
+          case PH_LM:
+            load_norm(P.x, nullptr, P.d);
+            prefetch_gain(P.attn_norm);
+            break;
+          default:
+            break;
         }
-        cand_warp_merge(v1, i1, v2);
-        if (lane == 0) sc->wcand[warp] = Cand{v1, i1, v2, 0};
-        cbar();
-        if (tid == 0) {
-          float a1 = -INFINITY, a2 = -INFINITY;
-          int ai = INT_MAX;
-          for (int w = 0; w < kConsumerWarps; ++w)
-            cand_merge(a1, ai, a2, sc->wcand[w].v1, sc->wcand[w].i1, sc->wcand[w].v2);
-          P.cand[c] = Cand{a1, ai, a2, 0};
-        }
-        if (!grid_sync()) return;
-        v1 = -INFINITY;
-        v2 = -INFINITY;
-        i1 = INT_MAX;
-        for (int cc = tid; cc < (int)gridDim.x; cc += kConsumerThreads) {
-          const float b1 = __ldcg(&P.cand[cc].v1);
-          const int bi = __ldcg(&P.cand[cc].i1);
-          const float b2 = __ldcg(&P.cand[cc].v2);
-          cand_merge(v1, i1, v2, b1, bi, b2);
-        }
-        cand_warp_merge(v1, i1, v2);
-        if (lane == 0) sc->wcand[warp] = Cand{v1, i1, v2, 0};
-        cbar();
-        if (tid == 0) {
-          float a1 = -INFINITY, a2 = -INFINITY;
-          int ai = INT_MAX;
-          for (int w = 0; w < kConsumerWarps; ++w)
-            cand_merge(a1, ai, a2, sc->wcand[w].v1, sc->wcand[w].i1, sc->wcand[w].v2);
-          sc->tok = ai;
-          sc->margin = a1 - a2;
-          if (c == 0) {
-            P.out_tokens[step] = ai;
-            if (P.margins_out) P.margins_out[step] = a1 - a2;
+        // ---- 2. tiles
+        if (kind == PH_ATTN) {
+          attention_dispatch(l, pos);
+        } else {
+          const int nseg = (P.E && (kind == PH_UP || kind == PH_DOWN)) ? 1 + P.top_k : 1;
+          int pnext = 0;
+          for (int si = 0; si < nseg; ++si) {
+            const SegDesc* sd;
+            int sk, voff = 0, pbase = 0, pstride, kjbase = 0;
+            if (kind == PH_QKV) { sd = &dc.at(l, 0); sk = SK_QKV; }
+            else if (kind == PH_O) { sd = &dc.at(l, 1); sk = SK_O; }
+            else if (kind == PH_LM) { sd = &dc.at(P.L, 0); sk = SK_LM; }
+            else if (kind == PH_UP) {
+              if (!P.E) { sd = &dc.at(l, 2); sk = SK_GU; }
+              else if (si == 0) { sd = &dc.at(l, 2); sk = SK_SGU; }
+              else { sd = &dc.at(l, 4 + re[si - 1]); sk = SK_EGU; pbase = pnext; rpb[si - 1] = pnext; }
+            } else {  // PH_DOWN
+              if (!P.E) { sd = &dc.at(l, 3); sk = SK_DOWN; }
+              else if (si == 0) { sd = &dc.at(l, 3); sk = SK_SDOWN; }
+              else {
+                sd = &dc.at(l, 4 + P.E + re[si - 1]);
+                sk = SK_EDOWN;
+                voff = P.ffs + (si - 1) * P.ffe;
+                kjbase = P.shp[SK_SDOWN].nk + (si - 1) * P.shp[SK_EDOWN].nk;
+              }
+            }
+            pstride = (kind == PH_DOWN && P.E) ? P.shp[SK_SDOWN].nk + P.top_k * P.shp[SK_EDOWN].nk
+                                               : P.shp[sk].nk;
+            run_segment(*sd, P.shp[sk], vec + voff / 2, pbase, pstride, kjbase);
+            pnext = pbase + sd->nrows * P.shp[sk].nk;
+            if (kind == PH_UP && P.E && si == 0) pnext = sd->nrows * P.shp[sk].nk;
           }
         }
         cbar();
-        next = sc->tok;
+        // ---- 3. epilogue
+        switch (kind) {
+          case PH_QKV:
+            epi_qkv(dc.at(l, 0), P.shp[SK_QKV].nk, l, pos);
+            break;
+          case PH_O:
+            epi_residual(dc.at(l, 1), P.shp[SK_O].nk, l == 0 ? erow : nullptr);
+            break;
+          case PH_UP:
+            if (!P.E) {
+              epi_swiglu(dc.at(l, 2), 0, P.shp[SK_GU].nk, 0, 1.0f);
+            } else {
+              epi_swiglu(dc.at(l, 2), 0, P.shp[SK_SGU].nk, 0, 1.0f);
+              for (int k = 0; k < P.top_k; ++k)
+                epi_swiglu(dc.at(l, 4 + re[k]), rpb[k], P.shp[SK_EGU].nk, P.ffs + k * P.ffe, rw[k]);
+            }
+            break;
+          case PH_DOWN:
+            epi_residual(dc.at(l, 3), P.E ? P.shp[SK_SDOWN].nk + P.top_k * P.shp[SK_EDOWN].nk : P.shp[SK_DOWN].nk,
+                         nullptr);
+            break;
+          case PH_LM:
+            epi_lm(dc.at(P.L, 0));
+            break;
+          default:
+            break;
+        }
+        if (!grid_sync()) return;
+      }
+      int next;
+      if (lm) {
+        next = pick_token();
         if (next == INT_MAX) {  // no finite logit
           if (tid == 0) record_error(P, kErrDevice, 5, step);
           return;
@@ -1168,6 +1265,58 @@ struct Consumer {
     }
     if (c == 0 && tid == 0) P.ctrl->final_token = tok;
   }
+
+  // LM-head epilogue: logits (optional copy out) and this CTA's greedy candidate.
+  __device__ void epi_lm(const SegDesc& dl) {
+    const int stride = P.shp[SK_LM].nk;
+    float v1 = -INFINITY, v2 = -INFINITY;
+    int i1 = INT_MAX;
+    for (int r = tid; r < dl.nrows; r += kConsumerThreads) {
+      const float y = row_sum(r, stride);
+      const int row = dl.row0 + r;
+      if (P.logits_out) P.logits_out[(size_t)step * P.V + row] = y;
+      cand_merge(v1, i1, v2, y, row, -INFINITY);
+    }
+    cand_warp_merge(v1, i1, v2);
+    if (lane == 0) sc->wcand[warp] = Cand{v1, i1, v2, 0};
+    cbar();
+    if (tid == 0) {
+      float a1 = -INFINITY, a2 = -INFINITY;
+      int ai = INT_MAX;
+      for (int w = 0; w < kConsumerWarps; ++w)
+        cand_merge(a1, ai, a2, sc->wcand[w].v1, sc->wcand[w].i1, sc->wcand[w].v2);
+      P.cand[blockIdx.x] = Cand{a1, ai, a2, 0};
+    }
+  }
+
+  // After the LM barrier: every CTA reduces all candidates the same way.
+  __device__ int pick_token() {
+    float v1 = -INFINITY, v2 = -INFINITY;
+    int i1 = INT_MAX;
+    for (int cc = tid; cc < (int)gridDim.x; cc += kConsumerThreads) {
+      const float b1 = __ldcg(&P.cand[cc].v1);
+      const int bi = __ldcg(&P.cand[cc].i1);
+      const float b2 = __ldcg(&P.cand[cc].v2);
+      cand_merge(v1, i1, v2, b1, bi, b2);
+    }
+    cand_warp_merge(v1, i1, v2);
+    if (lane == 0) sc->wcand[warp] = Cand{v1, i1, v2, 0};
+    cbar();
+    if (tid == 0) {
+      float a1 = -INFINITY, a2 = -INFINITY;
+      int ai = INT_MAX;
+      for (int w = 0; w < kConsumerWarps; ++w)
+        cand_merge(a1, ai, a2, sc->wcand[w].v1, sc->wcand[w].i1, sc->wcand[w].v2);
+      sc->tok = ai;
+      sc->margin = a1 - a2;
+      if (blockIdx.x == 0) {
+        P.out_tokens[step] = ai;
+        if (P.margins_out) P.margins_out[step] = a1 - a2;
+      }
+    }
+    cbar();
+    return sc->tok;
+  }
 };
 
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ Params P) {
@@ -1175,7 +1324,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   SmemCtl* sc = reinterpret_cast<SmemCtl*>(smem);
   float* part = reinterpret_cast<float*>(smem + smem_ctl_bytes());
   float* vec = part + kPartFloats;
-  unsigned char* ring = smem + smem_ring_offset(P.vec_floats);
+  SegDesc* dsm = reinterpret_cast<SegDesc*>(smem + smem_desc_offset(P.vec_floats));
+  unsigned char* ring = smem + smem_ring_offset(P.vec_floats, 4 * P.L + 1);
+  const SegDesc* dg = P.desc + (size_t)blockIdx.x * (P.L * P.slots + 1);
+  for (int i = threadIdx.x; i <= 4 * P.L; i += kThreads)
+    dsm[i] = (i < 4 * P.L) ? dg[(size_t)(i >> 2) * P.slots + (i & 3)] : dg[(size_t)P.L * P.slots];
+  const DescCache dc{dsm, dg, P.L, P.slots};
   if (threadIdx.x == 0) {
     for (int s = 0; s < P.n_stages; ++s) {
       mbar_init(&sc->full[s], 1);
@@ -1189,18 +1343,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   if (threadIdx.x >= kConsumerThreads) {
     const int lane = threadIdx.x - kConsumerThreads;
     if (lane < P.n_stages) {
-      Producer pr(P, sc, ring, lane);
+      Producer pr(P, sc, ring, lane, dc);
       pr.run();
     }
     return;
   }
-  Consumer cs(P, sc, part, vec, ring);
+  Consumer cs(P, sc, part, vec, ring, dc);
   cs.run();
 }
 
 // ---- host-side accessors used by the launcher
-int kernel_smem_bytes(int vec_floats, int n_stages, int stage_bytes) {
-  return smem_total(vec_floats, n_stages, stage_bytes);
+int kernel_smem_bytes(int vec_floats, int n_desc, int n_stages, int stage_bytes) {
+  return smem_total(vec_floats, n_desc, n_stages, stage_bytes);
 }
 int kernel_max_stages() { return kMaxStages; }
 const void* kernel_entry() { return reinterpret_cast<const void*>(&decode_kernel); }
