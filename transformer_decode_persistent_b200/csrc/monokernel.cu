@@ -533,6 +533,36 @@ __device__ __forceinline__ void tile_gemv_copyout(uint32_t w_s, uint32_t x_s, ui
   }
 }
 
+// K/V row slice of one lane (DPL fp16 head dims) from shared memory.
+template <int DPL>
+__device__ __forceinline__ uint2 lds_kv(uint32_t a) {
+  uint2 r = make_uint2(0u, 0u);
+  if constexpr (DPL == 4) asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(a));
+  else asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r.x) : "r"(a));
+  return r;
+}
+template <int DPL>
+__device__ __forceinline__ void kv_to_f32(uint2 r, float* f) {
+  const float2 a = h2f2(r.x);
+  f[0] = a.x;
+  f[1] = a.y;
+  if constexpr (DPL == 4) {
+    const float2 b = h2f2(r.y);
+    f[2] = b.x;
+    f[3] = b.y;
+  }
+}
+// This lane's share of q . k for one row.
+template <int DPL>
+__device__ __forceinline__ float qk_partial(const float* q, uint2 r) {
+  float f[DPL];
+  kv_to_f32<DPL>(r, f);
+  float t = q[0] * f[0];
+#pragma unroll
+  for (int e = 1; e < DPL; ++e) t = fmaf(q[e], f[e], t);
+  return t;
+}
+
 struct Consumer {
   const Params& P;
   SmemCtl* sc;
@@ -777,27 +807,16 @@ struct Consumer {
           float q[DPL];
 #pragma unroll
           for (int e = 0; e < DPL; ++e) q[e] = lds_f32(qsa + (uint32_t)(hh * DH + e) * 4u);
+          // All 32 rows of the stage are read; rows past the tile hold stale
+          // data whose scores only reach their own (masked) position.
           float part[kAttnSub];
 #pragma unroll
-          for (int jj = 0; jj < kAttnSub; ++jj) {
-            uint2 kr = make_uint2(0u, 0u);
-            if (jj < nsm) {
-              if constexpr (DPL == 4) asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(kr.x), "=r"(kr.y) : "r"(kt + jj * DH * 2) : "memory");
-              else asm("ld.shared.u32 %0, [%1];" : "=r"(kr.x) : "r"(kt + jj * DH * 2) : "memory");
-            } else if (jj == nsm && jj < nj) {
-              kr = kpos;
-            }
-            const float2 a = h2f2(kr.x);
-            float tt = q[0] * a.x;
-            tt = fmaf(q[1], a.y, tt);
-            if constexpr (DPL == 4) {
-              const float2 c2 = h2f2(kr.y);
-              tt = fmaf(q[2], c2.x, tt);
-              tt = fmaf(q[3], c2.y, tt);
-            }
-            part[jj] = tt;
+          for (int jj = 0; jj < kAttnSub; ++jj) part[jj] = qk_partial<DPL>(q, lds_kv<DPL>(kt + jj * DH * 2));
+          float a = transpose_reduce32(part, lane);
+          if (nsm < nj) {  // this token's own row, position nsm of the sub-block
+            const float own = warp_sum(qk_partial<DPL>(q, kpos));
+            if (lane == nsm) a = own;
           }
-          const float a = transpose_reduce32(part, lane);
           sts_f32(ssm + (uint32_t)(hh * kAttnSub + lane) * 4u, valid ? a : -INFINITY);
         }
       }
@@ -821,39 +840,33 @@ struct Consumer {
           m[hh] = mn;
         }
         const uint32_t vt = ring_s + (uint32_t)(sV * P.stage_bytes) + (uint32_t)(lane * DPL * 2);
-#pragma unroll 2
-        for (int jj = 0; jj < nj; jj += 2) {
-          uint2 va = make_uint2(0u, 0u), vb = make_uint2(0u, 0u);
-          if (jj < nsm) {
-            if constexpr (DPL == 4) asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(va.x), "=r"(va.y) : "r"(vt + jj * DH * 2) : "memory");
-            else asm("ld.shared.u32 %0, [%1];" : "=r"(va.x) : "r"(vt + jj * DH * 2) : "memory");
-          } else if (jj == nsm) {
-            va = vpos;
-          }
-          if (jj + 1 < nsm) {
-            if constexpr (DPL == 4) asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(vb.x), "=r"(vb.y) : "r"(vt + (jj + 1) * DH * 2) : "memory");
-            else asm("ld.shared.u32 %0, [%1];" : "=r"(vb.x) : "r"(vt + (jj + 1) * DH * 2) : "memory");
-          } else if (jj + 1 == nsm && jj + 1 < nj) {
-            vb = vpos;
-          }
+        // rows of the tile (positions 0 .. nsm-1), two at a time
+#pragma unroll 1
+        for (int jj = 0; jj < nsm; jj += 2) {
+          const int j2 = min(jj + 1, nsm - 1);
           float fa[DPL], fb[DPL];
-          {
-            const float2 a0 = h2f2(va.x), b0 = h2f2(vb.x);
-            fa[0] = a0.x; fa[1] = a0.y; fb[0] = b0.x; fb[1] = b0.y;
-            if constexpr (DPL == 4) {
-              const float2 a1 = h2f2(va.y), b1 = h2f2(vb.y);
-              fa[2] = a1.x; fa[3] = a1.y; fb[2] = b1.x; fb[3] = b1.y;
-            }
-          }
+          kv_to_f32<DPL>(lds_kv<DPL>(vt + jj * DH * 2), fa);
+          kv_to_f32<DPL>(lds_kv<DPL>(vt + j2 * DH * 2), fb);
+          const bool two = jj + 1 < nsm;  // warp-uniform
 #pragma unroll
           for (int hh = 0; hh < NH; ++hh) {
             const float pa = __shfl_sync(0xffffffffu, p[hh], jj);
-            const float pb = __shfl_sync(0xffffffffu, p[hh], (jj + 1) & 31);
+            const float pb = two ? __shfl_sync(0xffffffffu, p[hh], j2) : 0.f;
 #pragma unroll
             for (int e = 0; e < DPL; ++e) {
               acc[hh][e] = fmaf(pa, fa[e], acc[hh][e]);
               acc2[hh][e] = fmaf(pb, fb[e], acc2[hh][e]);
             }
+          }
+        }
+        if (nsm < nj) {  // this token's own row
+          float fv[DPL];
+          kv_to_f32<DPL>(vpos, fv);
+#pragma unroll
+          for (int hh = 0; hh < NH; ++hh) {
+            const float pv = __shfl_sync(0xffffffffu, p[hh], nsm);
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) acc[hh][e] = fmaf(pv, fv[e], acc[hh][e]);
           }
         }
       }
