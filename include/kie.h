@@ -155,8 +155,8 @@ kie_status kie_decode(kie_ctx* ctx, int n_tokens, int32_t* out_tokens,
  * The call allocates nothing and frees nothing. The kernel's per-launch
  * scratch lives in a 512 KiB array in the library's device image, which every
  * GPU that loads the library holds until the process exits. Models whose
- * scratch (about 4 bytes per residual, q/k/v, attention-output and FFN value,
- * plus attention partials) exceeds it are rejected with KIE_ERR_INVALID_ARG
+ * scratch (8 bytes per flagged value: two residual copies, q/k/v, attention
+ * output, FFN hidden; plus attention partials) exceeds it are rejected with KIE_ERR_INVALID_ARG
  * and a message giving both sizes. `out_tokens` must be device memory
  * ([n_tokens] int32, caller-owned); no logits, margins, forced tokens or trace.
  * The first call on a device looks up the array's device address (once per

@@ -183,8 +183,9 @@ def test_injected_barrier_fault_times_out_and_recovers(eng):
     p = S.make_prompt(SH, 0)
     eng.prefill(p)
     with pytest.raises(KieError) as ei:
-        # CTA 3 never arrives at grid barrier 4: every other CTA's wait runs out
-        eng.decode(4, timeout_ms=200, fault=(3, 4))
+        # CTA 3 never arrives at grid barrier 2 (the end of step 2): every
+        # other CTA's wait runs out
+        eng.decode(4, timeout_ms=200, fault=(3, 2))
     assert ei.value.status == -5 and "timeout" in str(ei.value)
     with pytest.raises(KieError) as ei:
         eng.decode(1)

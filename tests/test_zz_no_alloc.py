@@ -53,7 +53,7 @@ def test_static_scratch_decode_equals_decode_on_two_calls():
 
 
 def test_static_scratch_rejects_models_that_do_not_fit():
-    # 256 query heads of 128 dims over 64 KV heads need ~850 KB of scratch
+    # 256 query heads of 128 dims over 64 KV heads need about 1 MB of scratch
     s = S.Shape("wide-heads", n_layers=1, d_model=64, n_heads=256, n_kv_heads=64, head_dim=128,
                 ffn=64, vocab=100, max_ctx=1024)
     e = Engine(s)

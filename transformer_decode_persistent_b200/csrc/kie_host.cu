@@ -62,10 +62,10 @@ struct kie_ctx {
          *router = nullptr;
   __half *kcache = nullptr, *vcache = nullptr;
   float2* rope = nullptr;
-  float *x = nullptr, *qkv = nullptr, *o = nullptr, *h = nullptr, *apart = nullptr;
-  unsigned char* syncblk = nullptr;  // Ctrl + acnt[hk], cleared before every launch
+  float* apart = nullptr;
+  // Ctrl | acnt[L][hk] | flagged scratch (fx, fq, fo, fh, fcand), cleared before every launch
+  unsigned char* syncblk = nullptr;
   size_t syncblk_bytes = 0;
-  Cand* cand = nullptr;
   int *tok_dev = nullptr, *forced_dev = nullptr;
   float* margins_dev = nullptr;
   // state
@@ -240,6 +240,36 @@ struct Planner {
   }
 };
 
+// The region cleared before every launch: control block, attention arrival
+// counters and the flagged scratch words (see Params).
+struct SyncLayout {
+  size_t acnt, fx, fq, fo, fh, fcand, total;
+};
+
+SyncLayout sync_layout(const kie_config& k, int grid, int hbuf) {
+  auto a16 = [](size_t b) { return (b + 15) & ~(size_t)15; };
+  SyncLayout L{};
+  size_t off = a16(sizeof(Ctrl));
+  L.acnt = off;  off = a16(off + (size_t)k.n_layers * k.n_kv_heads * sizeof(unsigned));
+  L.fx = off;    off += (size_t)2 * k.d_model * 8;
+  L.fq = off;    off += (size_t)(k.n_heads + 2 * k.n_kv_heads) * k.head_dim * 8;
+  L.fo = off;    off += (size_t)k.n_heads * k.head_dim * 8;
+  L.fh = off;    off += (size_t)hbuf * 8;
+  L.fcand = off; off += (size_t)grid * 4 * 8;
+  L.total = off;
+  return L;
+}
+
+void set_sync_params(Params& P, unsigned char* base, const SyncLayout& L) {
+  P.ctrl = reinterpret_cast<Ctrl*>(base);
+  P.acnt = reinterpret_cast<unsigned*>(base + L.acnt);
+  P.fx = reinterpret_cast<unsigned long long*>(base + L.fx);
+  P.fq = reinterpret_cast<unsigned long long*>(base + L.fq);
+  P.fo = reinterpret_cast<unsigned long long*>(base + L.fo);
+  P.fh = reinterpret_cast<unsigned long long*>(base + L.fh);
+  P.fcand = reinterpret_cast<unsigned long long*>(base + L.fcand);
+}
+
 }  // namespace
 
 extern "C" {
@@ -358,16 +388,12 @@ kie_status kie_create(const kie_config* cfg, int device, kie_ctx** out) {
         cudaSuccess)
       return bail(fail(c, KIE_ERR_CUDA, "rope table upload failed"));
   }
-  if ((s = dalloc(c, &c->x, (size_t)d * 4)) ||
-      (s = dalloc(c, &c->qkv, (size_t)(hq + 2 * hk) * dh * 4)) ||
-      (s = dalloc(c, &c->o, (size_t)hq * dh * 4)) || (s = dalloc(c, &c->h, (size_t)c->hbuf * 4)) ||
-      (s = dalloc(c, &c->apart, (size_t)hq * c->max_chunks * (dh + 4) * 4)) ||
-      (s = dalloc(c, &c->cand, (size_t)c->grid * sizeof(Cand))) ||
+  if ((s = dalloc(c, &c->apart, (size_t)hq * c->max_chunks * (dh + 4) * 4)) ||
       (s = dalloc(c, &c->tok_dev, (size_t)k.max_ctx * 4)) ||
       (s = dalloc(c, &c->forced_dev, (size_t)k.max_ctx * 4)) ||
       (s = dalloc(c, &c->margins_dev, (size_t)k.max_ctx * 4)))
     return bail(s);
-  c->syncblk_bytes = sizeof(Ctrl) + (size_t)hk * sizeof(unsigned);
+  c->syncblk_bytes = sync_layout(k, c->grid, c->hbuf).total;
   if ((s = dalloc(c, &c->syncblk, c->syncblk_bytes))) return bail(s);
   if (cudaMemset(c->syncblk, 0, c->syncblk_bytes) != cudaSuccess)
     return bail(fail(c, KIE_ERR_CUDA, "memset failed"));
@@ -426,7 +452,7 @@ kie_status kie_get_info(const kie_ctx* c, kie_info* info) {
   info->n_stages = c->n_stages;
   info->stage_bytes = c->stage_bytes;
   info->smem_bytes = c->smem;
-  info->barriers_per_token = 5 * k.n_layers + 1;
+  info->barriers_per_token = 1;
   info->stream_bytes = c->stream_bytes;
   info->kv_bytes_per_pos = 2LL * k.n_layers * k.n_kv_heads * k.head_dim * 2;
   info->resident_bytes = (int64_t)c->tape_bytes;
@@ -800,10 +826,9 @@ kie_status launch(kie_ctx* c, const Run& r, cudaStream_t st) {
   P.embed = c->embed; P.attn_norm = c->attn_norm; P.mlp_norm = c->mlp_norm;
   P.final_norm = c->final_norm; P.router = c->router;
   P.kcache = c->kcache; P.vcache = c->vcache; P.rope = c->rope;
-  P.x = c->x; P.qkv = c->qkv; P.o = c->o; P.h = c->h; P.apart = c->apart;
-  P.ctrl = reinterpret_cast<Ctrl*>(c->syncblk);
-  P.acnt = reinterpret_cast<unsigned*>(c->syncblk + sizeof(Ctrl));
-  P.cand = c->cand; P.max_chunks = c->max_chunks;
+  P.apart = c->apart;
+  set_sync_params(P, c->syncblk, sync_layout(k, c->grid, c->hbuf));
+  P.max_chunks = c->max_chunks;
   P.pos0 = c->pos; P.n_steps = r.n_steps; P.first_token = r.first_token; P.lm_from_step = r.lm_from_step;
   P.forced = r.forced; P.out_tokens = r.out; P.logits_out = r.logits; P.margins_out = r.margins;
   P.timeout_ns = (unsigned long long)(r.timeout_ms ? r.timeout_ms : 1000u) * 1000000ull;
@@ -989,20 +1014,17 @@ unsigned char* g_static_ptr[kMaxDevices] = {};
 size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
 
 struct StaticLayout {
-  size_t x, qkv, o, h, apart, cand, sync, total;
+  size_t sync, sync_bytes, apart, total;
 };
 
 StaticLayout static_layout(const kie_ctx* c) {
   const kie_config& k = c->cfg;
   StaticLayout L{};
   size_t off = 0;
-  L.sync = off;  off += align256(sizeof(Ctrl) + (size_t)k.n_kv_heads * sizeof(unsigned));
-  L.x = off;     off += align256((size_t)k.d_model * 4);
-  L.qkv = off;   off += align256((size_t)(k.n_heads + 2 * k.n_kv_heads) * k.head_dim * 4);
-  L.o = off;     off += align256((size_t)k.n_heads * k.head_dim * 4);
-  L.h = off;     off += align256((size_t)c->hbuf * 4);
+  L.sync = off;
+  L.sync_bytes = sync_layout(k, c->grid, c->hbuf).total;
+  off += align256(L.sync_bytes);
   L.apart = off; off += align256((size_t)k.n_heads * c->max_chunks * (k.head_dim + 4) * 4);
-  L.cand = off;  off += align256((size_t)c->grid * sizeof(Cand));
   L.total = off;
   return L;
 }
@@ -1055,14 +1077,8 @@ extern "C" kie_status kie_decode_static(kie_ctx* c, int n, int32_t* out_tokens, 
   P.embed = c->embed; P.attn_norm = c->attn_norm; P.mlp_norm = c->mlp_norm;
   P.final_norm = c->final_norm; P.router = c->router;
   P.kcache = c->kcache; P.vcache = c->vcache; P.rope = c->rope;
-  P.x = reinterpret_cast<float*>(base + lay.x);
-  P.qkv = reinterpret_cast<float*>(base + lay.qkv);
-  P.o = reinterpret_cast<float*>(base + lay.o);
-  P.h = reinterpret_cast<float*>(base + lay.h);
   P.apart = reinterpret_cast<float*>(base + lay.apart);
-  P.ctrl = reinterpret_cast<Ctrl*>(base + lay.sync);
-  P.acnt = reinterpret_cast<unsigned*>(base + lay.sync + sizeof(Ctrl));
-  P.cand = reinterpret_cast<Cand*>(base + lay.cand);
+  set_sync_params(P, base + lay.sync, sync_layout(k, c->grid, c->hbuf));
   P.max_chunks = c->max_chunks;
   P.pos0 = c->pos; P.n_steps = n; P.first_token = c->pending; P.lm_from_step = 0;
   P.forced = nullptr; P.out_tokens = out_tokens; P.logits_out = nullptr; P.margins_out = nullptr;
@@ -1073,8 +1089,9 @@ extern "C" kie_status kie_decode_static(kie_ctx* c, int n, int32_t* out_tokens, 
   P.xplane = c->xplane;
   P.gbuf_off = c->gbuf_off;
   // the array keeps the previous call's contents: the barrier counter, the
-  // abort flag and the attention arrival counters must start at zero
-  CUDA_TRY(c, cudaMemsetAsync(base + lay.sync, 0, sizeof(Ctrl) + (size_t)k.n_kv_heads * sizeof(unsigned), st));
+  // abort flag, the attention arrival counters and the flagged words' epochs
+  // must start at zero
+  CUDA_TRY(c, cudaMemsetAsync(base + lay.sync, 0, lay.sync_bytes, st));
   void* args[] = {&P};
   cudaError_t e = cudaLaunchCooperativeKernel(kernel_entry(), dim3(c->grid), dim3(kThreads), args, (size_t)c->smem, st);
   if (e != cudaSuccess) {

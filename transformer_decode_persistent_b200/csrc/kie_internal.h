@@ -101,14 +101,18 @@ struct Params {
   __half* kcache;            // [L][hk][max_ctx][dh]
   __half* vcache;
   const float2* rope;        // [max_ctx][dh/2] (cos, sin)
-  // scratch
-  float* x;                  // [d] residual stream
-  float* qkv;                // [qkv_rows] raw q|k|v
-  float* o;                  // [hq*dh] attention output
-  float* h;                  // [hbuf] FFN hidden (dense: ff; MoE: ffs + top_k*ffe)
-  float* apart;              // attention partials [hq][max_chunks][dh + 4]
-  unsigned int* acnt;        // [hk] per-KV-head arrival counters
-  Cand* cand;                // [grid]
+  // Flagged scratch, zeroed before every launch. Each 64-bit word holds a
+  // float (low half) and the epoch of the phase that wrote it (high half);
+  // words are written and read as single 64-bit accesses, so a reader that
+  // sees the epoch it waits for also sees the value. Epoch of (step, layer l)
+  // = 1 + step * (L + 1) + l; the LM head of a step uses layer index L.
+  unsigned long long* fx;     // [2][d] residual stream after the output (0) / down (1) projection
+  unsigned long long* fq;     // [hq*dh | hk*dh | hk*dh] rotated scaled q | this token's k | v (fp16-rounded)
+  unsigned long long* fo;     // [hq*dh] attention output
+  unsigned long long* fh;     // [hbuf] FFN hidden (dense: ff; MoE: ffs + top_k*ffe)
+  unsigned long long* fcand;  // [grid][3] LM-head candidates: best value, its index, second value
+  float* apart;               // attention partials [hq][max_chunks][dh + 4]
+  unsigned int* acnt;         // [L][hk] per-layer, per-KV-head arrival counters (grow within a launch)
   Ctrl* ctrl;
   int max_chunks;
   // run

@@ -152,9 +152,37 @@ __device__ __forceinline__ unsigned ld_relaxed(const unsigned* p) {
   asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+// ---- flagged words: float value in the low half, writer's epoch in the high half
+__device__ __forceinline__ unsigned long long fpack(float v, unsigned ep) {
+  return ((unsigned long long)ep << 32) | __float_as_uint(v);
+}
+__device__ __forceinline__ void st_flag(unsigned long long* p, float v, unsigned ep) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(fpack(v, ep)) : "memory");
+}
+__device__ __forceinline__ void st_flag2(unsigned long long* p, float a, float b, unsigned ep) {
+  asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(fpack(a, ep)), "l"(fpack(b, ep))
+               : "memory");
+}
+__device__ __forceinline__ void ld_flag2(const unsigned long long* p, unsigned long long& a,
+                                         unsigned long long& b) {
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
+}
+__device__ __forceinline__ unsigned fepoch(unsigned long long w) { return (unsigned)(w >> 32); }
+__device__ __forceinline__ float fval(unsigned long long w) { return __uint_as_float((unsigned)w); }
 // consumer-only barrier (named barrier 1 over the 256 consumer threads)
 __device__ __forceinline__ void cbar() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
+}
+// consumer barrier that also ORs a predicate over the consumer threads, so
+// that all of them take the same branch on it
+__device__ __forceinline__ bool cbar_any(bool v) {
+  unsigned r;
+  asm volatile(
+      "{\n.reg .pred p, q;\nsetp.ne.u32 p, %1, 0;\nbar.red.or.pred q, 1, %2, p;\nselp.u32 %0, 1, 0, q;\n}"
+      : "=r"(r)
+      : "r"((unsigned)v), "n"(kConsumerThreads)
+      : "memory");
+  return r != 0;
 }
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -172,6 +200,13 @@ __device__ __forceinline__ float2 h2f2(unsigned u) {
   __half2 h;
   memcpy(&h, &u, sizeof(h));
   return __half22float2(h);
+}
+// two floats (already fp16-exact) as the bits of a half2
+__device__ __forceinline__ uint32_t f2h2(float a, float b) {
+  const __half2 h = __floats2half2_rn(a, b);
+  uint32_t u;
+  memcpy(&u, &h, 4);
+  return u;
 }
 
 // Explicit shared-memory loads by 32-bit shared address: the ring and the
@@ -572,6 +607,7 @@ struct Consumer {
   const int tid, warp, lane;
   unsigned tbase = 0;   // ring position (tiles consumed by the CTA so far)
   unsigned bar_no = 0;  // grid barriers passed
+  unsigned abase = 0;   // attention arrival-counter increments of the earlier steps of this launch
   int step = 0;
   unsigned route_round = 0;
 
@@ -592,6 +628,38 @@ struct Consumer {
     return t;
   }
 
+  __device__ __forceinline__ int ap_nchk(int pos) const { return attn_plan(pos, P.hk, gridDim.x).nchk; }
+
+  __device__ __forceinline__ unsigned epoch(int l) const { return 1u + (unsigned)step * (unsigned)(P.L + 1) + (unsigned)l; }
+
+  // Four flagged words at p (16-byte aligned) once they all carry epoch ep.
+  // Bounded: on abort or deadline it flags the CTA and returns zeros.
+  __device__ __forceinline__ float4 wait4(const unsigned long long* p, unsigned ep) {
+    unsigned long long a, b, c, d;
+    ld_flag2(p, a, b);
+    ld_flag2(p + 2, c, d);
+    if (fepoch(a) != ep || fepoch(b) != ep || fepoch(c) != ep || fepoch(d) != ep) {
+      const unsigned long long t0 = gtimer();
+      for (unsigned it = 1;; ++it) {
+        ld_flag2(p, a, b);
+        ld_flag2(p + 2, c, d);
+        if (fepoch(a) == ep && fepoch(b) == ep && fepoch(c) == ep && fepoch(d) == ep) break;
+        if ((it & 31) == 0) {
+          if (sc->abort || ld_relaxed(&P.ctrl->abort)) {
+            sc->abort = 1;
+            return make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          if (gtimer() - t0 > P.timeout_ns) {
+            record_error(P, kErrTimeout, 6, step);
+            sc->abort = 1;
+            return make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+      }
+    }
+    return make_float4(fval(a), fval(b), fval(c), fval(d));
+  }
+
   // The vector buffer holds an input vector split by halves of its 8-float
   // chunks: element i of chunk c (i < 4) at vec[4c + i], element 4 + i at
   // vec[xplane + 4c + i]. xv(i) is where the 4 elements from i (i % 4 == 0) go.
@@ -599,10 +667,10 @@ struct Consumer {
     return vec + ((i & 4) ? P.xplane : 0) + ((i >> 3) << 2);
   }
 
-  // vec = src (fp32, L2-resident scratch), n a multiple of 8
-  __device__ void load_vec(const float* src, int n) {
-    for (int i = tid * 4; i < n; i += kConsumerThreads * 4)
-      *reinterpret_cast<float4*>(xv(i)) = *reinterpret_cast<const float4*>(src + i);
+  // vec = the flagged vector src[0..n) of epoch ep (n a multiple of 8), once
+  // its producers have written it
+  __device__ void load_vec(const unsigned long long* src, unsigned ep, int n) {
+    for (int i = tid * 4; i < n; i += kConsumerThreads * 4) *reinterpret_cast<float4*>(xv(i)) = wait4(src + i, ep);
     cbar();
   }
 
@@ -616,14 +684,15 @@ struct Consumer {
     asm volatile("cp.async.commit_group;" ::: "memory");
   }
 
-  // vec = RMSNorm(src) * gain, src either fp32 (residual) or an fp16 embedding
-  // row; the gain was prefetched into the gain buffer by prefetch_gain.
-  __device__ void load_norm(const float* srcf, const __half* srch, int n) {
+  // vec = RMSNorm(src) * gain, src either the flagged residual stream of epoch
+  // ep or an fp16 embedding row; the gain was prefetched into the gain buffer
+  // by prefetch_gain.
+  __device__ void load_norm(const unsigned long long* srcf, unsigned ep, const __half* srch, int n) {
     float ss = 0.f;
     for (int i = tid * 4; i < n; i += kConsumerThreads * 4) {
       float4 v;
       if (srcf) {
-        v = *reinterpret_cast<const float4*>(srcf + i);
+        v = wait4(srcf + i, ep);
       } else {
         const uint2 raw = *reinterpret_cast<const uint2*>(srch + i);
         const float2 lo = h2f2(raw.x), hi = h2f2(raw.y);
@@ -764,8 +833,7 @@ struct Consumer {
       }
       sc->abort = ab;
     }
-    cbar();
-    return !sc->abort;
+    return !cbar_any(sc->abort != 0);
   }
 
   // One warp's share of one attention unit for a KV group of NH query heads:
@@ -915,20 +983,27 @@ struct Consumer {
       const int nh = (((g + 1) * hq + hk - 1) / hk) - h_lo;
       const int j0 = ch * ap.per, j1 = min(ap.T, j0 + ap.per);
       const int wj0 = j0 + vs * ap.pw, wj1 = min(j1, wj0 + ap.pw);
-      // this token's own row is not in the ring: fetch it now, use it last
+      // q of this group's heads and this token's own k/v row (not in the ring)
+      // come flagged from the q/k/v epilogues that produced them
+      const unsigned ep = epoch(l);
+      for (int i = tid * 4; i < nh * DH; i += kConsumerThreads * 4)
+        *reinterpret_cast<float4*>(qs + i) = wait4(P.fq + (size_t)h_lo * DH + i, ep);
       uint2 kpos = make_uint2(0u, 0u), vpos = make_uint2(0u, 0u);
       if (wj0 <= pos && pos < wj1) {
-        const size_t ro = ((size_t)(l * hk + g) * P.max_ctx + pos) * DH + lane * DPL;
+        const unsigned long long* kr = P.fq + (size_t)(hq + g) * DH + lane * DPL;
+        const unsigned long long* vr = P.fq + (size_t)(hq + hk + g) * DH + lane * DPL;
         if constexpr (DPL == 4) {
-          kpos = *reinterpret_cast<const uint2*>(P.kcache + ro);
-          vpos = *reinterpret_cast<const uint2*>(P.vcache + ro);
+          const float4 kf = wait4(kr, ep), vf = wait4(vr, ep);
+          kpos = make_uint2(f2h2(kf.x, kf.y), f2h2(kf.z, kf.w));
+          vpos = make_uint2(f2h2(vf.x, vf.y), f2h2(vf.z, vf.w));
         } else {
-          kpos.x = *reinterpret_cast<const unsigned*>(P.kcache + ro);
-          vpos.x = *reinterpret_cast<const unsigned*>(P.vcache + ro);
+          // two dims per lane: the aligned group of four holds this lane's pair
+          const float4 kf = wait4(kr - (lane & 1) * 2, ep), vf = wait4(vr - (lane & 1) * 2, ep);
+          kpos.x = (lane & 1) ? f2h2(kf.z, kf.w) : f2h2(kf.x, kf.y);
+          vpos.x = (lane & 1) ? f2h2(vf.z, vf.w) : f2h2(vf.x, vf.y);
         }
       }
-      for (int i = tid; i < nh * DH; i += kConsumerThreads) qs[i] = P.qkv[(size_t)h_lo * DH + i];
-      cbar();
+      if (cbar_any(sc->abort != 0)) return;
       switch (nh) {
         case 1: attn_warp<DH, 1>(ap, uo, vs, wj0, wj1, pos, kpos, vpos, qs, wp, sbuf); break;
         case 2: attn_warp<DH, 2>(ap, uo, vs, wj0, wj1, pos, kpos, vpos, qs, wp, sbuf); break;
@@ -956,8 +1031,9 @@ struct Consumer {
         const int h = h_lo + hh;
         if (ap.nchk == 1) {
           const float inv = 1.0f / Ls;
+          unsigned long long* ob = P.fo + (size_t)h * DH + lane * DPL;
 #pragma unroll
-          for (int e = 0; e < DPL; ++e) P.o[(size_t)h * DH + lane * DPL + e] = a[e] * inv;
+          for (int e = 0; e < DPL; e += 2) st_flag2(ob + e, a[e] * inv, a[e + 1] * inv, epoch(l));
         } else {
           float* gb = P.apart + ((size_t)h * P.max_chunks + ch) * WS;
           if (lane == 0) {
@@ -972,11 +1048,15 @@ struct Consumer {
         cbar();
         if (tid == 0) {
           unsigned old;
-          asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(P.acnt + g) : "memory");
+          asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;"
+                       : "=r"(old)
+                       : "l"(P.acnt + (size_t)l * hk + g)
+                       : "memory");
           sc->bcast = old;
         }
         cbar();
-        if (sc->bcast == (unsigned)(ap.nchk - 1)) {  // last CTA of this KV head: merge the chunks
+        // the counters grow through the launch: earlier steps added abase
+        if (sc->bcast == abase + (unsigned)(ap.nchk - 1)) {  // last CTA of this KV head: merge the chunks
           if (warp < nh) {
             const int h = h_lo + warp;
             const int nchk = ap.nchk;
@@ -1021,10 +1101,10 @@ struct Consumer {
             }
             Ls = warp_sum(Ls);
             const float inv = 1.0f / Ls;
+            unsigned long long* ob = P.fo + (size_t)h * DH + lane * DPL;
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) P.o[(size_t)h * DH + lane * DPL + e] = a[e] * inv;
+            for (int e = 0; e < DPL; e += 2) st_flag2(ob + e, a[e] * inv, a[e + 1] * inv, epoch(l));
           }
-          if (tid == 0) P.acnt[g] = 0u;
         }
       }
       cbar();  // qs / wp are reused by the next unit
@@ -1039,13 +1119,15 @@ struct Consumer {
 
   // q/k/v epilogue. The q/k/v rows are packed so that every CTA owns whole
   // RoPE pairs (dims i and i + dh/2 of one head are adjacent virtual rows), so
-  // RoPE is applied here: q is rotated and pre-scaled by 1/sqrt(dh) into the q
-  // scratch, k is rotated and appended (fp16) to the KV cache at `pos`, v is
-  // appended as is.
+  // RoPE is applied here: q is rotated and pre-scaled by 1/sqrt(dh), k is
+  // rotated and appended (fp16) to the KV cache at `pos`, v is appended as is;
+  // q and the fp16-rounded k and v are also published flagged for this step's
+  // attention.
   __device__ void epi_qkv(const SegDesc& sd, int stride, int l, int pos) {
     const int dh = P.dh, half = P.dh / 2, hq = P.hq, hk = P.hk;
     const float2* rp = P.rope + (size_t)pos * half;
     const float scale = 1.0f / sqrtf((float)dh);
+    const unsigned ep = epoch(l);
     for (int j = tid; j < sd.nrows / 2; j += kConsumerThreads) {
       const int r = sd.row0 + 2 * j;
       const int H = r / dh, pi = (r - H * dh) / 2;
@@ -1054,17 +1136,23 @@ struct Consumer {
         const float2 cs = rp[pi];
         const float a = ya * cs.x - yb * cs.y, b = ya * cs.y + yb * cs.x;
         if (H < hq) {
-          P.qkv[(size_t)H * dh + pi] = a * scale;
-          P.qkv[(size_t)H * dh + pi + half] = b * scale;
+          st_flag(P.fq + (size_t)H * dh + pi, a * scale, ep);
+          st_flag(P.fq + (size_t)H * dh + pi + half, b * scale, ep);
         } else {
           __half* k = P.kcache + ((size_t)(l * hk + (H - hq)) * P.max_ctx + pos) * dh;
-          k[pi] = __float2half_rn(a);
-          k[pi + half] = __float2half_rn(b);
+          const __half ka = __float2half_rn(a), kb = __float2half_rn(b);
+          k[pi] = ka;
+          k[pi + half] = kb;
+          st_flag(P.fq + (size_t)H * dh + pi, __half2float(ka), ep);
+          st_flag(P.fq + (size_t)H * dh + pi + half, __half2float(kb), ep);
         }
       } else {
         __half* v = P.vcache + ((size_t)(l * hk + (H - hq - hk)) * P.max_ctx + pos) * dh;
-        v[pi] = __float2half_rn(ya);
-        v[pi + half] = __float2half_rn(yb);
+        const __half va = __float2half_rn(ya), vb = __float2half_rn(yb);
+        v[pi] = va;
+        v[pi + half] = vb;
+        st_flag(P.fq + (size_t)H * dh + pi, __half2float(va), ep);
+        st_flag(P.fq + (size_t)H * dh + pi + half, __half2float(vb), ep);
       }
     }
     // the cache rows written here are read by TMA (async proxy) in later steps
@@ -1073,18 +1161,20 @@ struct Consumer {
 
   // residual epilogue: x[row] = xprev[row] + sum of partials. xprev is this
   // CTA's own copy of its rows (or the embedding row in the first layer).
-  __device__ void epi_residual(const SegDesc& sd, int stride, const __half* xprev_h) {
+  // The new rows are published flagged in the residual buffer `which`.
+  __device__ void epi_residual(const SegDesc& sd, int stride, const __half* xprev_h, int which, unsigned ep) {
+    unsigned long long* fx = P.fx + (size_t)which * P.d;
     for (int r = tid; r < sd.nrows; r += kConsumerThreads) {
       const int row = sd.row0 + r;
       const float xp = xprev_h ? __half2float(xprev_h[row]) : sc->xown[r];
       const float v = xp + row_sum(r, stride);
       sc->xown[r] = v;
-      P.x[row] = v;
+      st_flag(fx + row, v, ep);
     }
   }
 
   // SwiGLU epilogue over interleaved (gate, up) rows: h[hoff + row0/2 + j] = w * silu(g) * u
-  __device__ void epi_swiglu(const SegDesc& sd, int pbase, int stride, int hoff, float w) {
+  __device__ void epi_swiglu(const SegDesc& sd, int pbase, int stride, int hoff, float w, unsigned ep) {
     const int npairs = sd.nrows / 2;
     for (int j = tid; j < npairs; j += kConsumerThreads) {
       float yg = 0.f, yu = 0.f;
@@ -1092,7 +1182,7 @@ struct Consumer {
         yg += part[pbase + (2 * j) * stride + k];
         yu += part[pbase + (2 * j + 1) * stride + k];
       }
-      P.h[hoff + sd.row0 / 2 + j] = w * silu(yg) * yu;
+      st_flag(P.fh + hoff + sd.row0 / 2 + j, w * silu(yg) * yu, ep);
     }
   }
 
@@ -1140,12 +1230,14 @@ struct Consumer {
     ++route_round;
   }
 
-  // The per-token step as a sequence of phases separated by grid barriers:
-  // per layer q/k/v, attention, output projection, FFN up (gate/up or routed
-  // experts), FFN down; then the LM head when the step samples. Every phase
-  // reads its input vector, runs its tiles through the one run_segment call
-  // site (one inlined copy of the GEMV code keeps the instruction cache warm),
-  // then runs its epilogue.
+  // The per-token step as a sequence of phases: per layer q/k/v, attention,
+  // output projection, FFN up (gate/up or routed experts), FFN down; then the
+  // LM head when the step samples. Every phase waits for the flagged input it
+  // reads (so it starts as soon as that input's producers are done, with no
+  // grid-wide barrier between phases), runs its tiles through the one
+  // run_segment call site (one inlined copy of the GEMV code keeps the
+  // instruction cache warm), then runs its epilogue, which publishes its
+  // output flagged.
   enum PhaseKind { PH_QKV = 0, PH_ATTN = 1, PH_O = 2, PH_UP = 3, PH_DOWN = 4, PH_LM = 5 };
 
   __device__ void run() {
@@ -1170,15 +1262,15 @@ struct Consumer {
         // ---- 1. input vector
         switch (kind) {
           case PH_QKV:
-            if (l == 0) load_norm(nullptr, erow, P.d);
-            else load_norm(P.x, nullptr, P.d);
+            if (l == 0) load_norm(nullptr, 0u, erow, P.d);
+            else load_norm(P.fx + P.d, epoch(l - 1), nullptr, P.d);
             prefetch_gain(P.mlp_norm + (size_t)l * P.d);
             break;
           case PH_O:
-            load_vec(P.o, P.hq * P.dh);
+            load_vec(P.fo, epoch(l), P.hq * P.dh);
             break;
           case PH_UP:
-            load_norm(P.x, nullptr, P.d);
+            load_norm(P.fx, epoch(l), nullptr, P.d);
             if (l + 1 < P.L) prefetch_gain(P.attn_norm + (size_t)(l + 1) * P.d);
             else prefetch_gain(lm ? P.final_norm : P.attn_norm);
             if (P.E) {
@@ -1191,10 +1283,10 @@ struct Consumer {
             }
             break;
           case PH_DOWN:
-            load_vec(P.h, P.E ? P.ffs + P.top_k * P.ffe : P.ff);
+            load_vec(P.fh, epoch(l), P.E ? P.ffs + P.top_k * P.ffe : P.ff);
             break;
           case PH_LM:
-            load_norm(P.x, nullptr, P.d);
+            load_norm(P.fx + P.d, epoch(P.L - 1), nullptr, P.d);
             prefetch_gain(P.attn_norm);
             break;
           default:
@@ -1240,20 +1332,20 @@ struct Consumer {
             epi_qkv(dc.at(l, 0), P.shp[SK_QKV].nk, l, pos);
             break;
           case PH_O:
-            epi_residual(dc.at(l, 1), P.shp[SK_O].nk, l == 0 ? erow : nullptr);
+            epi_residual(dc.at(l, 1), P.shp[SK_O].nk, l == 0 ? erow : nullptr, 0, epoch(l));
             break;
           case PH_UP:
             if (!P.E) {
-              epi_swiglu(dc.at(l, 2), 0, P.shp[SK_GU].nk, 0, 1.0f);
+              epi_swiglu(dc.at(l, 2), 0, P.shp[SK_GU].nk, 0, 1.0f, epoch(l));
             } else {
-              epi_swiglu(dc.at(l, 2), 0, P.shp[SK_SGU].nk, 0, 1.0f);
+              epi_swiglu(dc.at(l, 2), 0, P.shp[SK_SGU].nk, 0, 1.0f, epoch(l));
               for (int k = 0; k < P.top_k; ++k)
-                epi_swiglu(dc.at(l, 4 + re[k]), rpb[k], P.shp[SK_EGU].nk, P.ffs + k * P.ffe, rw[k]);
+                epi_swiglu(dc.at(l, 4 + re[k]), rpb[k], P.shp[SK_EGU].nk, P.ffs + k * P.ffe, rw[k], epoch(l));
             }
             break;
           case PH_DOWN:
             epi_residual(dc.at(l, 3), P.E ? P.shp[SK_SDOWN].nk + P.top_k * P.shp[SK_EDOWN].nk : P.shp[SK_DOWN].nk,
-                         nullptr);
+                         nullptr, 1, epoch(l));
             break;
           case PH_LM:
             epi_lm(dc.at(P.L, 0));
@@ -1261,11 +1353,12 @@ struct Consumer {
           default:
             break;
         }
-        if (!grid_sync()) return;
+        if (cbar_any(sc->abort != 0)) return;
       }
       int next;
       if (lm) {
         next = pick_token();
+        if (cbar_any(sc->abort != 0)) return;
         if (next == INT_MAX) {  // no finite logit
           if (tid == 0) record_error(P, kErrDevice, 5, step);
           return;
@@ -1275,6 +1368,11 @@ struct Consumer {
         next = P.forced ? P.forced[step] : -1;
       }
       tok = next;
+      // one grid barrier per step: it orders this step's KV-cache appends
+      // before the next step's bulk copies of them (the phases within a step
+      // wait on the flagged words they read instead)
+      if (!grid_sync()) return;
+      if (ap_nchk(pos) > 1) abase += (unsigned)ap_nchk(pos);
     }
     if (c == 0 && tid == 0) P.ctrl->final_token = tok;
   }
@@ -1298,19 +1396,19 @@ struct Consumer {
       int ai = INT_MAX;
       for (int w = 0; w < kConsumerWarps; ++w)
         cand_merge(a1, ai, a2, sc->wcand[w].v1, sc->wcand[w].i1, sc->wcand[w].v2);
-      P.cand[blockIdx.x] = Cand{a1, ai, a2, 0};
+      unsigned long long* cb = P.fcand + (size_t)blockIdx.x * 4;
+      st_flag2(cb, a1, __int_as_float(ai), epoch(P.L));
+      st_flag2(cb + 2, a2, 0.f, epoch(P.L));
     }
   }
 
-  // After the LM barrier: every CTA reduces all candidates the same way.
+  // Every CTA reduces all CTAs' flagged candidates the same way.
   __device__ int pick_token() {
     float v1 = -INFINITY, v2 = -INFINITY;
     int i1 = INT_MAX;
     for (int cc = tid; cc < (int)gridDim.x; cc += kConsumerThreads) {
-      const float b1 = __ldcg(&P.cand[cc].v1);
-      const int bi = __ldcg(&P.cand[cc].i1);
-      const float b2 = __ldcg(&P.cand[cc].v2);
-      cand_merge(v1, i1, v2, b1, bi, b2);
+      const float4 cv = wait4(P.fcand + (size_t)cc * 4, epoch(P.L));
+      cand_merge(v1, i1, v2, cv.x, __float_as_int(cv.y), cv.z);
     }
     cand_warp_merge(v1, i1, v2);
     if (lane == 0) sc->wcand[warp] = Cand{v1, i1, v2, 0};
