@@ -134,6 +134,13 @@ bool is_device_ptr(const void* p) {
 // g >= 4 (the input vector chunk is reused across g rows) with the fewest
 // chunks; GU kinds need an even g so (gate, up) pairs share a tile.
 SegShape choose_shape(int K, bool pairs, int stage_bytes) {
+  // Preferred: column blocks of 512 halves (two 16-byte chunks per lane, up to
+  // kMaxRowsWide rows) or of 768 halves (three chunks, up to 8 rows): the
+  // kernel's register-blocked tile GEMVs for these widths take any row count.
+  if (K % 512 == 0 && stage_bytes / 1024 >= 4)
+    return SegShape{K, std::min(kMaxRowsWide, stage_bytes / 1024), K / 512, 512};
+  if (K % 768 == 0 && stage_bytes / 1536 >= 4)
+    return SegShape{K, std::min(kMaxRowsPerTile, stage_bytes / 1536), K / 768, 768};
   // First choice: the fewest column blocks that give at least 4 rows per
   // tile. A split into more blocks wins when its chunks divide evenly over the
   // 32 lanes (kc a multiple of 256 halves, so the kernel's copy-out GEMV

@@ -16,8 +16,9 @@ constexpr int kConsumerThreads = kConsumerWarps * 32;  // named barrier 1 spans 
 constexpr int kThreads = kConsumerThreads + 32;        // + one producer (TMA) warp
 constexpr int kRingStages = 2 * kConsumerWarps;        // ring stages per CTA (2 per consumer warp)
 constexpr int kMaxStageBytes = 16384;                  // upper bound of one stage (one weight tile)
-constexpr int kMaxRowsPerTile = 8;                     // rows of one tile (register-blocked)
-constexpr int kPartFloats = 1024;                      // per-CTA partial-sum slots per phase
+constexpr int kMaxRowsPerTile = 8;                     // rows of one tile in general (register-blocked)
+constexpr int kMaxRowsWide = 13;                       // rows of a tile 512 halves wide
+constexpr int kPartFloats = 1280;                      // per-CTA partial-sum slots per phase
 constexpr int kMaxHeadsPerGroup = 4;                   // query heads per KV head (GQA)
 constexpr int kMaxTopK = 4;                            // routed experts per token
 constexpr int kAttnSub = 32;                           // positions per attention sub-block

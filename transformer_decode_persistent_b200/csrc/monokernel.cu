@@ -310,6 +310,27 @@ __device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
   return v[0];
 }
 
+// N values per lane (N a power of two up to 16) summed over the warp: lane l
+// ends with the warp total of value (l mod N). Butterfly on the low lane bits,
+// then plain sums over the remaining bits.
+template <int N>
+__device__ __forceinline__ float transpose_reduce(float (&v)[N], int lane) {
+#pragma unroll
+  for (int o = N / 2; o >= 1; o /= 2) {
+    const bool up = lane & o;
+#pragma unroll
+    for (int k = 0; k < o; ++k) {
+      const float send = up ? v[k] : v[k + o];
+      const float keep = up ? v[k + o] : v[k];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  float r = v[0];
+#pragma unroll
+  for (int o = N; o < 32; o *= 2) r += __shfl_xor_sync(0xffffffffu, r, o);
+  return r;
+}
+
 // ---------------------------------------------------------------- errors
 
 __device__ void record_error(const Params& P, int code, int where, int step) {
@@ -470,7 +491,6 @@ struct Producer {
   }
 
   __device__ void run() {
-    const int c = blockIdx.x;
     bool ok = true;
     unsigned route_round = 0;
     for (step = 0; ok && step < P.n_steps; ++step) {
@@ -536,36 +556,38 @@ __device__ __forceinline__ void tile_gemv(uint32_t w_s, uint32_t x_s, uint32_t x
   }
 }
 
-// Same product for full tiles of G rows and 32*CPL chunks: the lane's whole
-// share of the tile is first copied to registers, the stage is released at
-// once (so its next bulk copy starts about a GEMV earlier), then the math runs
-// from registers.
-template <int G, int CPL>
-__device__ __forceinline__ void tile_gemv_copyout(uint32_t w_s, uint32_t x_s, uint32_t xpb, int lane, float* part,
-                                                  int pidx0, int pstride, uint64_t* empty) {
+// Tile of g <= GM rows x 32*CPL chunks (rows past g are skipped): the lane's
+// share is copied to registers and the stage released at once, then two
+// accumulators per row, and one butterfly turns the rows' lane partials into
+// lane r holding row r's sum.
+template <int GM, int CPL>
+__device__ __forceinline__ void tile_gemv_rows(uint32_t w_s, uint32_t x_s, uint32_t xpb, int lane, float* part,
+                                               int pidx0, int pstride, uint64_t* empty, int g) {
   constexpr int nch = CPL * 32;
-  uint4 wr[G][CPL];
+  constexpr int NP = GM <= 8 ? 8 : 16;
+  uint4 wr[GM][CPL];
 #pragma unroll
   for (int k = 0; k < CPL; ++k)
 #pragma unroll
-    for (int r = 0; r < G; ++r) wr[r][k] = lds_u4(w_s + (uint32_t)(r * nch + lane + 32 * k) * 16u);
+    for (int r = 0; r < GM; ++r)
+      wr[r][k] = r < g ? lds_u4(w_s + (uint32_t)(r * nch + lane + 32 * k) * 16u) : make_uint4(0u, 0u, 0u, 0u);
   __syncwarp();
   if (lane == 0) mbar_arrive(empty);
-  float acc[G][2];
+  float acc[GM][2];
 #pragma unroll
-  for (int r = 0; r < G; ++r) acc[r][0] = acc[r][1] = 0.f;
+  for (int r = 0; r < GM; ++r) acc[r][0] = acc[r][1] = 0.f;
 #pragma unroll
   for (int k = 0; k < CPL; ++k) {
     const uint32_t xa = x_s + (uint32_t)(lane + 32 * k) * 16u;
     const float4 a = lds_f4(xa), b = lds_f4(xa + xpb);
 #pragma unroll
-    for (int r = 0; r < G; ++r) acc[r][k & 1] = dot8(wr[r][k], a, b, acc[r][k & 1]);
+    for (int r = 0; r < GM; ++r) acc[r][k & 1] = dot8(wr[r][k], a, b, acc[r][k & 1]);
   }
+  float v[NP];
 #pragma unroll
-  for (int r = 0; r < G; ++r) {
-    const float v = warp_sum(acc[r][0] + acc[r][1]);
-    if (lane == r) part[pidx0 + r * pstride] = v;
-  }
+  for (int r = 0; r < NP; ++r) v[r] = r < GM ? acc[r][0] + acc[r][1] : 0.f;
+  const float t = transpose_reduce<NP>(v, lane);
+  if (lane < g) part[pidx0 + lane * pstride] = t;
 }
 
 // K/V row slice of one lane (DPL fp16 head dims) from shared memory.
@@ -746,21 +768,10 @@ struct Consumer {
       const uint32_t xpb = (uint32_t)P.xplane * 4u;
       const int p0 = pbase + gi * sh.g * pstride + kjbase + kj;
       uint64_t* em = &sc->empty[s];
-      bool done = false;
-      if (gp == sh.g && (nch & 31) == 0) {
-        done = true;
-        switch (gp * 16 + (nch >> 5)) {
-          case 8 * 16 + 1: tile_gemv_copyout<8, 1>(w, xs, xpb, lane, part, p0, pstride, em); break;
-          case 8 * 16 + 3: tile_gemv_copyout<8, 3>(w, xs, xpb, lane, part, p0, pstride, em); break;
-          case 6 * 16 + 3: tile_gemv_copyout<6, 3>(w, xs, xpb, lane, part, p0, pstride, em); break;
-          case 4 * 16 + 5: tile_gemv_copyout<4, 5>(w, xs, xpb, lane, part, p0, pstride, em); break;
-          case 5 * 16 + 5: tile_gemv_copyout<5, 5>(w, xs, xpb, lane, part, p0, pstride, em); break;
-          case 4 * 16 + 6: tile_gemv_copyout<4, 6>(w, xs, xpb, lane, part, p0, pstride, em); break;
-          case 6 * 16 + 4: tile_gemv_copyout<6, 4>(w, xs, xpb, lane, part, p0, pstride, em); break;
-          case 7 * 16 + 4: tile_gemv_copyout<7, 4>(w, xs, xpb, lane, part, p0, pstride, em); break;
-          default: done = false;
-        }
-      }
+      bool done = true;
+      if (nch == 64 && gp <= 13) tile_gemv_rows<13, 2>(w, xs, xpb, lane, part, p0, pstride, em, gp);
+      else if (nch == 96 && gp <= 8) tile_gemv_rows<8, 3>(w, xs, xpb, lane, part, p0, pstride, em, gp);
+      else done = false;
       if (!done) {
         switch (gp) {
           case 1: tile_gemv<1>(w, xs, xpb, nch, lane, part, p0, pstride, em); break;
@@ -908,22 +919,33 @@ struct Consumer {
           m[hh] = mn;
         }
         const uint32_t vt = ring_s + (uint32_t)(sV * P.stage_bytes) + (uint32_t)(lane * DPL * 2);
-        // rows of the tile (positions 0 .. nsm-1), two at a time
-#pragma unroll 1
-        for (int jj = 0; jj < nsm; jj += 2) {
-          const int j2 = min(jj + 1, nsm - 1);
-          float fa[DPL], fb[DPL];
-          kv_to_f32<DPL>(lds_kv<DPL>(vt + jj * DH * 2), fa);
-          kv_to_f32<DPL>(lds_kv<DPL>(vt + j2 * DH * 2), fb);
-          const bool two = jj + 1 < nsm;  // warp-uniform
+        // p of every position to shared memory (the score slots), read back
+        // four at a time as broadcasts; all 32 rows of the V stage are
+        // loaded at once and rows past the tile are masked out by select
 #pragma unroll
-          for (int hh = 0; hh < NH; ++hh) {
-            const float pa = __shfl_sync(0xffffffffu, p[hh], jj);
-            const float pb = two ? __shfl_sync(0xffffffffu, p[hh], j2) : 0.f;
+        for (int hh = 0; hh < NH; ++hh) sts_f32(ssm + (uint32_t)(hh * kAttnSub + lane) * 4u, p[hh]);
+        __syncwarp();
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) {
-              acc[hh][e] = fmaf(pa, fa[e], acc[hh][e]);
-              acc2[hh][e] = fmaf(pb, fb[e], acc2[hh][e]);
+        for (int j4 = 0; j4 < kAttnSub; j4 += 4) {
+          float4 pv[NH];
+#pragma unroll
+          for (int hh = 0; hh < NH; ++hh) pv[hh] = lds_f4(ssm + (uint32_t)(hh * kAttnSub + j4) * 4u);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int j = j4 + u;
+            float f[DPL];
+            kv_to_f32<DPL>(lds_kv<DPL>(vt + j * DH * 2), f);
+            const bool in = j < nsm;
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) f[e] = in ? f[e] : 0.f;
+#pragma unroll
+            for (int hh = 0; hh < NH; ++hh) {
+              const float pj = u == 0 ? pv[hh].x : u == 1 ? pv[hh].y : u == 2 ? pv[hh].z : pv[hh].w;
+#pragma unroll
+              for (int e = 0; e < DPL; ++e) {
+                if (u & 1) acc2[hh][e] = fmaf(pj, f[e], acc2[hh][e]);
+                else acc[hh][e] = fmaf(pj, f[e], acc[hh][e]);
+              }
             }
           }
         }
@@ -968,7 +990,7 @@ struct Consumer {
   __device__ void attention(int l, int pos) {
     constexpr int DPL = DH / 32;   // head dims per lane
     constexpr int WS = DH + 4;     // partial record: m, l, pad, pad, acc[DH]
-    const int hk = P.hk, hq = P.hq, G = gridDim.x, ns = P.n_stages;
+    const int hk = P.hk, hq = P.hq, G = gridDim.x;
     const AttnPlan ap = attn_plan(pos, hk, G);
     const int nu = attn_units_of(ap, blockIdx.x, G);
     const int vs = (int)((warp + kConsumerWarps - (int)(tbase % kConsumerWarps)) % kConsumerWarps);
