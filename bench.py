@@ -217,7 +217,8 @@ def main():
     ap.add_argument("--decode", type=int, default=None, help="override decode length (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--trace", action="store_true", help="also run a traced decode (barrier stall share)")
+    ap.add_argument("--trace", action="store_true",
+                    help="also run traced decodes: step-barrier wait share, per-step time of the first and last 64 steps")
     args = ap.parse_args()
 
     import synthetic as S
@@ -324,14 +325,30 @@ def main():
 
     stall = None
     if args.trace and rank == 0:
-        cap = min(n, 64) * info["barriers_per_token"]
-        tr = torch.zeros((info["grid"], cap, 2), dtype=torch.int64, device="cuda")
-        eng.reset()
-        eng.prefill(prompt)
-        eng.decode(min(n, 64), trace=tr)
-        t = tr.cpu().numpy().astype(np.float64)
+        # globaltimer stamps of the step barrier (arrival, release) per CTA:
+        # the share of time CTAs wait in it, and the per-step time from one
+        # release to the next, over the first and the last 64 steps
+        m = min(n, 64)
+        cap = m * info["barriers_per_token"]
+
+        def traced(pos, tok):
+            tr = torch.zeros((info["grid"], cap, 2), dtype=torch.int64, device="cuda")
+            eng.rewind(pos, tok)
+            r = eng.decode(m, trace=tr)
+            return tr.cpu().numpy().astype(np.float64), r["tokens"]
+
+        stall = {}
+        if n > m:  # the last steps first: rewind only moves back from the current position
+            toks = out.cpu().numpy()
+            t2, _ = traced(P - 1 + n - m, int(toks[n - m - 1]))
+            rel2 = np.median(t2[:, :, 1], axis=0)
+            stall["step_us_last"] = float(np.diff(rel2).mean() / 1000.0)
+        t, _ = traced(P - 1, int(prompt[-1]))
         span = t[:, :, 1].max() - t[:, :, 0].min()
-        stall = float(((t[:, :, 1] - t[:, :, 0]).sum(axis=1) / span).mean())
+        stall["barrier_wait_share"] = float(((t[:, :, 1] - t[:, :, 0]).sum(axis=1) / span).mean())
+        rel = np.median(t[:, :, 1], axis=0)
+        stall["step_us_first"] = float(np.diff(rel).mean() / 1000.0)
+        stall["steps_averaged"] = m
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -364,7 +381,7 @@ def main():
             "cpu_baseline": cpu,
         }
         if stall is not None:
-            line["barrier_stall_share"] = stall
+            line["trace"] = stall
         print(json.dumps(line), flush=True)
     if ws > 1:
         dist.barrier()
