@@ -27,6 +27,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import re
 import os
 import statistics
 import subprocess
@@ -52,10 +53,15 @@ def _peaks():
 
 
 def _kernel_hash() -> str:
+    """Hash of the decode kernel's code (comments and whitespace removed), so
+    DRAM counters stay attached to the code they were taken on."""
     h = hashlib.sha256()
     for f in ("monokernel.cu", "kie_internal.h"):
-        with open(os.path.join(ROOT, "transformer_decode_persistent_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "transformer_decode_persistent_b200", "csrc", f)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update(re.sub(r"\s+", " ", src).strip().encode())
     return h.hexdigest()[:16]
 
 

@@ -1,33 +1,38 @@
 // Persistent batch-1 decode kernel for B200 (sm_100a).
 //
-// One cooperative launch runs n whole decode steps: "MatMul, attention,
-// normalization and sampling" inside one GPU-resident program that feeds each
-// new token back to itself without returning to the host ("メモリの壁を打破する：
-// 標準的なGPUで3,000 tokens/sの推論を実現する", section "1. The Monokernel Runtime").
-// At batch 1 the step is bound by moving every active weight from HBM once per
-// token (same page, section "ボトルネック：計算量ではなくメモリ帯域幅"), so the
-// kernel is organised around keeping HBM busy:
+// One cooperative launch runs n whole decode steps: every matrix product, the
+// attention, the normalisations and the token choice stay inside one
+// GPU-resident program that feeds each new token back to itself without a
+// return to the host ("メモリの壁を打破する：標準的なGPUで3,000 tokens/sの推論を
+// 実現する", section "1. The Monokernel Runtime"). At batch 1 a step is bound by
+// moving every active weight from HBM once per token (same page, section
+// "ボトルネック：計算量ではなくメモリ帯域幅"), so the kernel is organised around
+// keeping HBM busy and the dependency chain short:
 //
 //  * One CTA per SM. Each CTA owns a contiguous region of a packed "weight
 //    tape" that holds, in execution order, its slice of every matrix of one
 //    decode step (see kie_internal.h for the tile format).
-//  * Warp 8 of each CTA is a producer: one lane streams the CTA's tape into a
-//    ring of shared-memory stages with TMA bulk copies (cp.async.bulk, L2
-//    evict-first), completion tracked by mbarriers. It never waits for the
-//    grid barriers, so the next phase's (and next layer's) weights are already
-//    in flight while the current phase reduces and synchronises.
-//  * Warps 0-7 are consumers: GEMV on each tile against the fp32 input vector
+//  * Warp 7 of each CTA is the producer: lanes 0..13 each own one of 14
+//    shared-memory ring stages and stream the CTA's tape tiles (and attention
+//    K/V rows) into it with TMA bulk copies (cp.async.bulk, L2 evict-first),
+//    completion tracked by mbarriers. It never waits on the consumers' data
+//    dependencies, so the next phase's weights are in flight while the current
+//    phase finishes.
+//  * Warps 0-6 are consumers: GEMV on each tile against the fp32 input vector
 //    held in shared memory (fp16 weights, fp32 FMA), RMSNorm (recomputed by
-//    every CTA from the L2-resident residual), RoPE, split-K attention over the
-//    fp16 KV cache, SwiGLU, residual adds, the LM head and a greedy argmax.
-//  * Dependent phases are joined by a grid barrier (monotonic arrival counter,
-//    release/acquire at GPU scope) with a %globaltimer deadline: the
-//    synchronisation cost the pages name ("マイクロ秒が失われる場所") is paid in a
-//    few hundred ns, and hidden behind the producer's prefetch.
+//    every CTA), RoPE, split-K attention over the fp16 KV cache, SwiGLU,
+//    residual adds, the LM head and a greedy argmax.
+//  * Phases exchange data through flagged 64-bit words (value and the epoch of
+//    the phase that wrote it): a phase waits only for the words it reads, so
+//    there is no grid-wide barrier between phases. One grid barrier per step
+//    orders the step's KV-cache appends before the next step's bulk copies.
+//    This is where the per-operation synchronisation cost that the pages
+//    name (same page, section "マイクロ秒が失われる場所") is removed.
 //
-// Every wait (grid barrier, ring stages, routing hand-off) is bounded: on a
-// deadline the kernel records KIE_ERR_TIMEOUT in the control block, raises an
-// abort flag that all CTAs poll, lets in-flight bulk copies land, and returns.
+// Every wait (flagged words, step barrier, ring stages, routing hand-off) is
+// bounded: on a deadline the kernel records KIE_ERR_TIMEOUT in the control
+// block, raises an abort flag that all CTAs poll, lets in-flight bulk copies
+// land, and returns.
 #include <cuda_fp16.h>
 #include <float.h>
 #include <limits.h>
@@ -805,7 +810,7 @@ struct Consumer {
     return y;
   }
 
-  // Grid-wide barrier between dependent phases. Returns false if the run aborted.
+  // Grid-wide barrier, once per step (see run). Returns false if the run aborted.
   __device__ bool grid_sync() {
     cbar();
     if (tid == 0) {
