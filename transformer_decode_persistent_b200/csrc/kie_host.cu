@@ -864,8 +864,8 @@ kie_status launch(kie_ctx* c, const Run& r, cudaStream_t st) {
   if (ctl.err) {
     c->poisoned = true;
     static const char* where[] = {"?", "grid barrier", "ring stage (full)", "ring stage (empty)",
-                                  "expert routing hand-off", "device check"};
-    const int w = (ctl.err_where >= 1 && ctl.err_where <= 5) ? ctl.err_where : 0;
+                                  "expert routing hand-off", "device check", "flagged input wait"};
+    const int w = (ctl.err_where >= 1 && ctl.err_where <= 6) ? ctl.err_where : 0;
     return fail(c, (kie_status)ctl.err, "device %s at %s (cta %d, step %d); context poisoned",
                 ctl.err == KIE_ERR_TIMEOUT ? "timeout" : "check failed", where[w], ctl.err_cta,
                 ctl.err_step);
@@ -897,7 +897,7 @@ kie_status kie_prefill(kie_ctx* c, const int32_t* tokens, int n, void* stream) {
                 c->cfg.max_ctx);
   cudaSetDevice(c->device);
   cudaStream_t st = (cudaStream_t)stream;
-  const int kChunk = 8192;  // bounds the barrier counter of one launch
+  const int kChunk = 8192;  // bounds the barrier counter and the flag epochs of one launch
   const int32_t new_pending = tokens[n - 1];
   size_t i0 = 0;
   const int32_t pos_before = c->pos, pend_before = c->pending;

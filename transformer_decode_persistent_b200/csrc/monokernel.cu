@@ -174,7 +174,7 @@ __device__ __forceinline__ void ld_flag2(const unsigned long long* p, unsigned l
 }
 __device__ __forceinline__ unsigned fepoch(unsigned long long w) { return (unsigned)(w >> 32); }
 __device__ __forceinline__ float fval(unsigned long long w) { return __uint_as_float((unsigned)w); }
-// consumer-only barrier (named barrier 1 over the 256 consumer threads)
+// consumer-only barrier (named barrier 1 over the 224 consumer threads)
 __device__ __forceinline__ void cbar() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
 }
