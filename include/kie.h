@@ -1,10 +1,11 @@
 /*
  * kie.h -- C ABI of the batch-1 decode engine (libkie.so), NVIDIA B200 (sm_100a).
  *
- * What the library computes. The pages describe a "persistent monokernel": one
- * GPU-resident program that runs the whole per-token decode step -- MatMul,
- * attention, normalization and sampling -- and hands each new token back to
- * itself without returning control to the CPU ("メモリの壁を打破する：標準的なGPUで
+ * What the library computes. The pages describe a persistent single-kernel
+ * runtime: one GPU-resident program that runs the whole per-token decode step
+ * (every matrix product, the attention, the normalisations and the token
+ * choice) and hands each new token back to itself without returning control
+ * to the CPU ("メモリの壁を打破する：標準的なGPUで
  * 3,000 tokens/sの推論を実現する", section "1. The Monokernel Runtime"; "Kog、より深い
  * GPU最適化でAI推論を高速化できると賭ける", section "KogがGPU推論の最適化をさらに
  * 深める理由"). At batch 1 the step is bound by streaming every active weight from

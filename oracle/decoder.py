@@ -6,8 +6,9 @@ module. The GPU engine never calls it and shares no code with it; the two meet
 only in the seeded inputs of the ``synthetic`` module.
 
 What it computes. The pages describe one persistent GPU program that performs
-the whole per-token decode step -- "MatMul, attention, normalization and
-sampling" -- and emits output tokens one by one without returning to the host
+the whole per-token decode step (the matrix products, attention, normalisations
+and the token choice) and emits output tokens one by one without returning to
+the host
 ("メモリの壁を打破する：標準的なGPUで3,000 tokens/sの推論を実現する", section
 "1. The Monokernel Runtime"; "Kog、より深いGPU最適化でAI推論を高速化できると賭ける",
 section "KogがGPU推論の最適化をさらに深める理由"). Batch-1 decode with a KV cache
@@ -29,9 +30,9 @@ math; the readings taken (all listed in the design notes) are:
   value minus the second-largest value (0 on a tie).
 * No biases, no QK-norm, no logit scaling. Weights are fp16 and widened to
   fp64 at use.
-* The KV cache is fp16: the workload descriptions fix it ("KV cache fp16",
-  "prefilled into an fp16 KV cache") and the method attends "over an FP16 KV
-  cache". So K (after RoPE) and V are rounded to fp16 (round to nearest even)
+* The KV cache is fp16: the workload descriptions fix it (the cache, and the
+  prompt prefilled into it, are fp16) and the method's attention reads an
+  fp16 cache. So K (after RoPE) and V are rounded to fp16 (round to nearest even)
   when they enter the cache, in both the incremental and the full-sequence
   form; every other step stays in fp64. ``kv_fp16=False`` keeps them
   unrounded (for diagnosis).
