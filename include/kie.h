@@ -195,6 +195,50 @@ int32_t kie_pending(const kie_ctx* ctx);
 /* Fill *info for a context whose weights are loaded. Errors: INVALID_ARG, STATE. */
 kie_status kie_get_info(const kie_ctx* ctx, kie_info* info);
 
+/* Tile shape of one kind of matrix segment: K input columns cut into nk
+ * column blocks of kc halves (K = nk * kc); a tile holds up to g rows of one
+ * column block and is one bulk copy into a ring stage. */
+typedef struct {
+  int32_t K, g, nk, kc;
+} kie_seg_shape;
+
+/* One CTA's share of one matrix: rows [row0, row0 + nrows) of the matrix's
+ * packed row order, stored at byte offset `off` of the weight tape (nrows * K
+ * fp16 values as tiles of the kind's shape). Packed row order: q/k/v rows are
+ * [wq; wk; wv] with each head's dims ordered 0, dh/2, 1, dh/2 + 1, ... (RoPE
+ * pairs adjacent); gate/up rows alternate gate_0, up_0, gate_1, up_1, ...;
+ * other matrices keep their own row order. */
+typedef struct {
+  int64_t off;
+  int32_t row0, nrows;
+} kie_seg_range;
+
+typedef struct {
+  int32_t slots;          /* ranges per layer: 4 dense; 4 + 2 * n_experts MoE      */
+  int32_t ranges_per_cta; /* n_layers * slots + 1                                 */
+  int64_t tape_bytes;     /* size of the packed weight tape                       */
+  kie_seg_shape shapes[9]; /* by kind: 0 q/k/v, 1 o, 2 gate/up, 3 down, 4 shared
+                              gate/up, 5 expert gate/up, 6 shared down, 7 expert
+                              down, 8 LM head; kinds the model lacks are zero     */
+} kie_plan_info;
+
+/* The weight-tape plan the engine uses for `grid` CTAs with ring stages of
+ * `stage_bytes` (kie_get_info reports both for a real context): tile shapes,
+ * and per CTA c, layer l and slot s the range ranges[c * ranges_per_cta +
+ * l * slots + s] (slot 0 q/k/v, 1 o, 2 gate/up or shared gate/up, 3 down or
+ * shared down, 4 + e expert e's gate/up, 4 + E + e expert e's down), with the
+ * LM head's range last. The tape holds each CTA's ranges contiguously in that
+ * order; the o and down ranges of a CTA are the same residual rows in every
+ * layer. Pure host arithmetic: needs no GPU and allocates no device memory.
+ * `ranges` may be NULL (then only *info is filled); otherwise it is a
+ * caller-owned array of `capacity` entries, at least grid * ranges_per_cta.
+ * Errors: INVALID_ARG for a shape kie_create would reject, grid < 1,
+ * stage_bytes < 4096 or not a multiple of 16, a plan that needs more
+ * per-CTA partial sums than the kernel holds, or too small a capacity
+ * (message from kie_last_error(NULL)). */
+kie_status kie_plan(const kie_config* cfg, int32_t grid, int32_t stage_bytes, kie_plan_info* info,
+                    kie_seg_range* ranges, int64_t capacity);
+
 #ifdef __cplusplus
 }
 #endif

@@ -48,6 +48,10 @@ def test_struct_layouts_match_header():
     assert ctypes.sizeof(K.kie_tensor) == 40
     assert ctypes.sizeof(K.kie_decode_opts) == 56
     assert ctypes.sizeof(K.kie_info) == 56
+    # plan: shape 4*4; range 8 + 2*4; info 2*4 + 8 + 9*16
+    assert ctypes.sizeof(K.kie_seg_shape) == 16
+    assert ctypes.sizeof(K.kie_seg_range) == 16
+    assert ctypes.sizeof(K.kie_plan_info) == 160
 
 
 def _cfg(**kw):

@@ -217,16 +217,13 @@ __global__ void pack_rows_kernel(const unsigned long long* __restrict__ src,
 namespace {
 
 struct Planner {
-  kie_ctx* c;
   const kie_config& k;
   int G;
   int slots;
   std::vector<SegDesc> desc;  // [G][L*slots + 1]
-  std::vector<size_t> cta_bytes;
 
-  Planner(kie_ctx* ctx) : c(ctx), k(ctx->cfg), G(ctx->grid), slots(ctx->slots) {
+  Planner(const kie_config& cfg, int grid, int nslots) : k(cfg), G(grid), slots(nslots) {
     desc.assign((size_t)G * (k.n_layers * slots + 1), SegDesc{0, 0, 0});
-    cta_bytes.assign(G, 0);
   }
 
   // rows of kind over the (virtual) row space, split into G near-equal ranges;
@@ -246,6 +243,116 @@ struct Planner {
     (void)kind;
   }
 };
+
+// Segment kind of descriptor slot `slot` of layer l (l == L: the LM head).
+int kind_of(const kie_config& k, int l, int slot) {
+  if (l == k.n_layers) return SK_LM;
+  if (slot == 0) return SK_QKV;
+  if (slot == 1) return SK_O;
+  if (k.n_experts == 0) return slot == 2 ? SK_GU : SK_DOWN;
+  if (slot == 2) return SK_SGU;
+  if (slot == 3) return SK_SDOWN;
+  return slot < 4 + k.n_experts ? SK_EGU : SK_EDOWN;
+}
+
+// The weight-tape plan for `grid` CTAs with ring stages of `sb` bytes: the
+// tile shape of every segment kind, each CTA's row range of every matrix
+// (desc, [grid][L*slots + 1]) and its byte offset in the tape (each CTA's
+// region contiguous, segments in execution order). Pure host arithmetic.
+struct Plan {
+  SegShape shp[SK_COUNT] = {};
+  std::vector<SegDesc> desc;
+  size_t tape_bytes = 0;
+  int slots = 0;
+};
+
+kie_status make_plan(kie_ctx* c, const kie_config& k, int G, int sb, Plan& plan) {
+  const bool moe = k.n_experts > 0;
+  const int d = k.d_model, hq = k.n_heads, hk = k.n_kv_heads, dh = k.head_dim, L = k.n_layers;
+  const int ffs = k.ffn_shared, ffe = k.ffn_expert;
+  SegShape* shp = plan.shp;
+  shp[SK_QKV] = balance_rows(choose_shape(d, false, sb), (hq + 2 * hk) * dh, 2, false, G);
+  shp[SK_O] = balance_rows(choose_shape(hq * dh, false, sb), d, 1, false, G);
+  shp[SK_LM] = balance_rows(choose_shape(d, false, sb), k.vocab, 1, false, G);
+  if (!moe) {
+    shp[SK_GU] = balance_rows(choose_shape(d, true, sb), 2 * k.ffn, 2, true, G);
+    shp[SK_DOWN] = balance_rows(choose_shape(k.ffn, false, sb), d, 1, false, G);
+  } else {
+    shp[SK_SGU] = balance_rows(choose_shape(d, true, sb), 2 * ffs, 2, true, G);
+    shp[SK_EGU] = balance_rows(choose_shape(d, true, sb), 2 * ffe, 2, true, G);
+    shp[SK_SDOWN] = balance_rows(choose_shape(ffs, false, sb), d, 1, false, G);
+    shp[SK_EDOWN] = balance_rows(choose_shape(ffe, false, sb), d, 1, false, G);
+  }
+  for (int i = 0; i < SK_COUNT; ++i)
+    if (shp[i].K && shp[i].g < 1)
+      return fail(c, KIE_ERR_INVALID_ARG, "no tile shape of %d columns fits a %d-byte ring stage", shp[i].K, sb);
+
+  // row assignment
+  plan.slots = slots_per_layer(moe ? k.n_experts : 0);
+  Planner pl(k, G, plan.slots);
+  for (int l = 0; l < L; ++l) {
+    const int rot = (int)(((long long)l * 53) % G);
+    pl.assign(l, 0, SK_QKV, (hq + 2 * hk) * dh, rot);
+    // the output and down projections own the same residual rows in every
+    // layer (no rotation): each CTA keeps its rows in shared memory
+    pl.assign(l, 1, SK_O, d, 0);
+    if (!moe) {
+      pl.assign(l, 2, SK_GU, 2 * k.ffn, (rot + 31) % G);
+      pl.assign(l, 3, SK_DOWN, d, 0);
+    } else {
+      pl.assign(l, 2, SK_SGU, 2 * ffs, (rot + 31) % G);
+      pl.assign(l, 3, SK_SDOWN, d, 0);
+      for (int e = 0; e < k.n_experts; ++e) {
+        pl.assign(l, 4 + e, SK_EGU, 2 * ffe, (rot + 97 + 7 * e) % G);
+        pl.assign(l, 4 + k.n_experts + e, SK_EDOWN, d, 0);
+      }
+    }
+  }
+  pl.assign(L, 0, SK_LM, k.vocab, 0);
+
+  const int slots = plan.slots;
+  const int per_cta = L * slots + 1;
+  // partial-slot capacity per phase
+  {
+    int worst = 0;
+    for (int ci = 0; ci < G; ++ci) {
+      const SegDesc* D = &pl.desc[(size_t)ci * per_cta];
+      for (int l = 0; l < L; ++l) {
+        const SegDesc* Dl = D + (size_t)l * slots;
+        worst = std::max(worst, Dl[0].nrows * shp[SK_QKV].nk);
+        worst = std::max(worst, Dl[1].nrows * shp[SK_O].nk);
+        if (!moe) {
+          worst = std::max(worst, Dl[2].nrows * shp[SK_GU].nk);
+          worst = std::max(worst, Dl[3].nrows * shp[SK_DOWN].nk);
+        } else {
+          int eg = 0;
+          for (int e = 0; e < k.n_experts; ++e) eg = std::max(eg, Dl[4 + e].nrows);
+          worst = std::max(worst, Dl[2].nrows * shp[SK_SGU].nk + k.top_k * eg * shp[SK_EGU].nk);
+          worst = std::max(worst, Dl[3].nrows * (shp[SK_SDOWN].nk + k.top_k * shp[SK_EDOWN].nk));
+        }
+      }
+      worst = std::max(worst, D[(size_t)L * slots].nrows * shp[SK_LM].nk);
+    }
+    if (worst > kPartFloats)
+      return fail(c, KIE_ERR_INVALID_ARG, "a CTA would hold %d partial sums (max %d)", worst, kPartFloats);
+  }
+
+  // tape offsets: each CTA's region contiguous, segments in execution order
+  size_t off = 0;
+  for (int ci = 0; ci < G; ++ci) {
+    for (int l = 0; l <= L; ++l) {
+      const int ns = (l == L) ? 1 : slots;
+      for (int slot = 0; slot < ns; ++slot) {
+        SegDesc& sd = pl.desc[(size_t)ci * per_cta + (size_t)l * slots + slot];
+        sd.off = off;
+        off += (size_t)sd.nrows * shp[kind_of(k, l, slot)].K * 2;
+      }
+    }
+  }
+  plan.tape_bytes = off;
+  plan.desc = std::move(pl.desc);
+  return KIE_OK;
+}
 
 // The region cleared before every launch: control block, attention arrival
 // counters and the flagged scratch words (see Params).
@@ -277,15 +384,8 @@ void set_sync_params(Params& P, unsigned char* base, const SyncLayout& L) {
   P.fcand = reinterpret_cast<unsigned long long*>(base + L.fcand);
 }
 
-}  // namespace
-
-extern "C" {
-
-kie_status kie_create(const kie_config* cfg, int device, kie_ctx** out) {
-  g_create_error.clear();
-  if (!cfg || !out) return fail(nullptr, KIE_ERR_INVALID_ARG, "null argument");
-  *out = nullptr;
-  const kie_config& k = *cfg;
+// Shape checks shared by kie_create and kie_plan (messages via kie_last_error(NULL)).
+kie_status validate_config(const kie_config& k) {
   const bool moe = k.n_experts > 0;
   if (k.n_layers < 1 || k.d_model < 8 || k.n_heads < 1 || k.n_kv_heads < 1 || k.head_dim < 2 ||
       k.vocab < 2 || k.max_ctx < 1)
@@ -315,6 +415,20 @@ kie_status kie_create(const kie_config* cfg, int device, kie_ctx** out) {
   if (!(k.rms_eps >= 0.f) || !(k.rope_theta > 0.f))
     return fail(nullptr, KIE_ERR_INVALID_ARG, "bad rms_eps / rope_theta");
 
+  return KIE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kie_status kie_create(const kie_config* cfg, int device, kie_ctx** out) {
+  g_create_error.clear();
+  if (!cfg || !out) return fail(nullptr, KIE_ERR_INVALID_ARG, "null argument");
+  *out = nullptr;
+  const kie_config& k = *cfg;
+  const bool moe = k.n_experts > 0;
+  if (kie_status vs = validate_config(k)) return vs;
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
     cudaGetLastError();
@@ -450,6 +564,32 @@ kie_status kie_rewind(kie_ctx* c, int32_t pos, int32_t pending) {
   return KIE_OK;
 }
 
+kie_status kie_plan(const kie_config* cfg, int32_t grid, int32_t stage_bytes, kie_plan_info* info,
+                    kie_seg_range* ranges, int64_t capacity) {
+  g_create_error.clear();
+  if (!cfg || !info) return fail(nullptr, KIE_ERR_INVALID_ARG, "null argument");
+  if (kie_status vs = validate_config(*cfg)) return vs;
+  if (grid < 1) return fail(nullptr, KIE_ERR_INVALID_ARG, "grid %d < 1", grid);
+  if (stage_bytes < 4096 || stage_bytes % 16)
+    return fail(nullptr, KIE_ERR_INVALID_ARG, "stage_bytes %d: at least 4096 and a multiple of 16", stage_bytes);
+  Plan plan;
+  if (kie_status ps = make_plan(nullptr, *cfg, grid, stage_bytes, plan)) return ps;
+  const int per_cta = cfg->n_layers * plan.slots + 1;
+  info->slots = plan.slots;
+  info->ranges_per_cta = per_cta;
+  info->tape_bytes = (int64_t)plan.tape_bytes;
+  for (int i = 0; i < SK_COUNT; ++i)
+    info->shapes[i] = kie_seg_shape{plan.shp[i].K, plan.shp[i].g, plan.shp[i].nk, plan.shp[i].kc};
+  if (ranges) {
+    if (capacity < (int64_t)plan.desc.size())
+      return fail(nullptr, KIE_ERR_INVALID_ARG, "ranges holds %lld entries, the plan has %zu",
+                  (long long)capacity, plan.desc.size());
+    for (size_t i = 0; i < plan.desc.size(); ++i)
+      ranges[i] = kie_seg_range{(int64_t)plan.desc[i].off, plan.desc[i].row0, plan.desc[i].nrows};
+  }
+  return KIE_OK;
+}
+
 kie_status kie_get_info(const kie_ctx* c, kie_info* info) {
   if (!c || !info) return KIE_ERR_INVALID_ARG;
   if (!c->loaded) return KIE_ERR_STATE;
@@ -568,101 +708,20 @@ kie_status kie_load_weights(kie_ctx* c, const kie_tensor* tensors, int n, void* 
     }
   }
 
-  // segment shapes
+  // segment shapes, row assignment and tape offsets
   const int ffs = k.ffn_shared, ffe = k.ffn_expert;
-  {
-    const int G = c->grid, sb = c->stage_bytes;
-    c->shp[SK_QKV] = balance_rows(choose_shape(d, false, sb), (hq + 2 * hk) * dh, 2, false, G);
-    c->shp[SK_O] = balance_rows(choose_shape(hq * dh, false, sb), d, 1, false, G);
-    c->shp[SK_LM] = balance_rows(choose_shape(d, false, sb), k.vocab, 1, false, G);
-    if (!moe) {
-      c->shp[SK_GU] = balance_rows(choose_shape(d, true, sb), 2 * k.ffn, 2, true, G);
-      c->shp[SK_DOWN] = balance_rows(choose_shape(k.ffn, false, sb), d, 1, false, G);
-    } else {
-      c->shp[SK_SGU] = balance_rows(choose_shape(d, true, sb), 2 * ffs, 2, true, G);
-      c->shp[SK_EGU] = balance_rows(choose_shape(d, true, sb), 2 * ffe, 2, true, G);
-      c->shp[SK_SDOWN] = balance_rows(choose_shape(ffs, false, sb), d, 1, false, G);
-      c->shp[SK_EDOWN] = balance_rows(choose_shape(ffe, false, sb), d, 1, false, G);
-    }
-  }
-
-  // row assignment
-  Planner pl(c);
   const int G = c->grid;
-  for (int l = 0; l < L; ++l) {
-    const int rot = (int)(((long long)l * 53) % G);
-    pl.assign(l, 0, SK_QKV, (hq + 2 * hk) * dh, rot);
-    // the output and down projections own the same residual rows in every
-    // layer (no rotation): each CTA keeps its rows in shared memory
-    pl.assign(l, 1, SK_O, d, 0);
-    if (!moe) {
-      pl.assign(l, 2, SK_GU, 2 * k.ffn, (rot + 31) % G);
-      pl.assign(l, 3, SK_DOWN, d, 0);
-    } else {
-      pl.assign(l, 2, SK_SGU, 2 * ffs, (rot + 31) % G);
-      pl.assign(l, 3, SK_SDOWN, d, 0);
-      for (int e = 0; e < k.n_experts; ++e) {
-        pl.assign(l, 4 + e, SK_EGU, 2 * ffe, (rot + 97 + 7 * e) % G);
-        pl.assign(l, 4 + k.n_experts + e, SK_EDOWN, d, 0);
-      }
-    }
+  Plan plan;
+  if ((s = make_plan(c, k, G, c->stage_bytes, plan))) {
+    dfree(c, staging);
+    return s;
   }
-  pl.assign(L, 0, SK_LM, k.vocab, 0);
-
-  auto kind_of = [&](int l, int slot) -> int {
-    if (l == L) return SK_LM;
-    if (slot == 0) return SK_QKV;
-    if (slot == 1) return SK_O;
-    if (!moe) return slot == 2 ? SK_GU : SK_DOWN;
-    if (slot == 2) return SK_SGU;
-    if (slot == 3) return SK_SDOWN;
-    return slot < 4 + k.n_experts ? SK_EGU : SK_EDOWN;
-  };
+  for (int i = 0; i < SK_COUNT; ++i) c->shp[i] = plan.shp[i];
+  auto kind_of = [&](int l, int slot) -> int { return ::kind_of(k, l, slot); };
   const int per_cta = L * c->slots + 1;
-  // partial-slot capacity per phase
-  {
-    int worst = 0;
-    for (int ci = 0; ci < G; ++ci) {
-      const SegDesc* D = &pl.desc[(size_t)ci * per_cta];
-      for (int l = 0; l < L; ++l) {
-        const SegDesc* Dl = D + (size_t)l * c->slots;
-        worst = std::max(worst, Dl[0].nrows * c->shp[SK_QKV].nk);
-        worst = std::max(worst, Dl[1].nrows * c->shp[SK_O].nk);
-        if (!moe) {
-          worst = std::max(worst, Dl[2].nrows * c->shp[SK_GU].nk);
-          worst = std::max(worst, Dl[3].nrows * c->shp[SK_DOWN].nk);
-        } else {
-          int eg = 0, ed = 0;
-          for (int e = 0; e < k.n_experts; ++e) {
-            eg = std::max(eg, Dl[4 + e].nrows);
-            ed = std::max(ed, Dl[4 + k.n_experts + e].nrows);
-          }
-          worst = std::max(worst, Dl[2].nrows * c->shp[SK_SGU].nk + k.top_k * eg * c->shp[SK_EGU].nk);
-          worst = std::max(worst, Dl[3].nrows * (c->shp[SK_SDOWN].nk + k.top_k * c->shp[SK_EDOWN].nk));
-        }
-      }
-      worst = std::max(worst, D[(size_t)L * c->slots].nrows * c->shp[SK_LM].nk);
-    }
-    if (worst > kPartFloats) {
-      dfree(c, staging);
-      return fail(c, KIE_ERR_INVALID_ARG, "a CTA would hold %d partial sums (max %d)", worst, kPartFloats);
-    }
-  }
-
-  // tape offsets: each CTA's region contiguous, segments in execution order
-  size_t off = 0;
-  for (int ci = 0; ci < G; ++ci) {
-    for (int l = 0; l <= L; ++l) {
-      const int ns = (l == L) ? 1 : c->slots;
-      for (int slot = 0; slot < ns; ++slot) {
-        SegDesc& sd = pl.desc[(size_t)ci * per_cta + (size_t)l * c->slots + slot];
-        sd.off = off;
-        off += (size_t)sd.nrows * c->shp[kind_of(l, slot)].K * 2;
-      }
-    }
-  }
-  c->tape_bytes = off;
-  if ((s = dalloc(c, &c->tape, off))) {
+  const std::vector<SegDesc>& desc = plan.desc;
+  c->tape_bytes = plan.tape_bytes;
+  if ((s = dalloc(c, &c->tape, c->tape_bytes))) {
     dfree(c, staging);
     return s;
   }
@@ -734,7 +793,7 @@ kie_status kie_load_weights(kie_ctx* c, const kie_tensor* tensors, int n, void* 
       const SegShape& sh = c->shp[kind_of(l, slot)];
       // resolve two base pointers per slot once (even/odd rows for GU kinds)
       for (int ci = 0; ci < G; ++ci) {
-        const SegDesc& sd = pl.desc[(size_t)ci * per_cta + (size_t)l * c->slots + slot];
+        const SegDesc& sd = desc[(size_t)ci * per_cta + (size_t)l * c->slots + slot];
         const int ngroups = (sd.nrows + sh.g - 1) / sh.g;
         for (int gi = 0; gi < ngroups; ++gi) {
           const int gp = std::min(sh.g, sd.nrows - gi * sh.g);
@@ -761,8 +820,8 @@ kie_status kie_load_weights(kie_ctx* c, const kie_tensor* tensors, int n, void* 
   dfree(c, dsrc); dfree(c, ddst); dfree(c, dn);
 
   // descriptors and the small tensors kept outside the tape
-  if ((s = dalloc(c, &c->desc, pl.desc.size() * sizeof(SegDesc)))) return s;
-  CUDA_TRY(c, cudaMemcpyAsync(c->desc, pl.desc.data(), pl.desc.size() * sizeof(SegDesc),
+  if ((s = dalloc(c, &c->desc, desc.size() * sizeof(SegDesc)))) return s;
+  CUDA_TRY(c, cudaMemcpyAsync(c->desc, desc.data(), desc.size() * sizeof(SegDesc),
                               cudaMemcpyHostToDevice, st));
   if ((s = dalloc(c, &c->embed, (size_t)k.vocab * d * 2)) ||
       (s = dalloc(c, &c->attn_norm, (size_t)L * d * 2)) || (s = dalloc(c, &c->mlp_norm, (size_t)L * d * 2)) ||

@@ -21,7 +21,7 @@ STATUS = {0: "KIE_OK", -1: "KIE_ERR_INVALID_ARG", -2: "KIE_ERR_STATE", -3: "KIE_
 
 EXPORTS = ["kie_create", "kie_load_weights", "kie_prefill", "kie_decode", "kie_decode_static",
            "kie_rewind", "kie_reset", "kie_destroy", "kie_last_error", "kie_position",
-           "kie_pending", "kie_get_info"]
+           "kie_pending", "kie_get_info", "kie_plan"]
 
 
 class KieError(RuntimeError):
@@ -56,6 +56,22 @@ class kie_info(ctypes.Structure):
                 ("stream_bytes", "kv_bytes_per_pos", "resident_bytes", "launches")]
 
 
+class kie_seg_shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("K", "g", "nk", "kc")]
+
+
+class kie_seg_range(ctypes.Structure):
+    _fields_ = [("off", ctypes.c_int64), ("row0", ctypes.c_int32), ("nrows", ctypes.c_int32)]
+
+
+class kie_plan_info(ctypes.Structure):
+    _fields_ = [("slots", ctypes.c_int32), ("ranges_per_cta", ctypes.c_int32),
+                ("tape_bytes", ctypes.c_int64), ("shapes", kie_seg_shape * 9)]
+
+
+SEG_KINDS = ("qkv", "o", "gate_up", "down", "shared_gate_up", "expert_gate_up", "shared_down",
+             "expert_down", "lm_head")
+
 _lib = None
 
 
@@ -84,8 +100,10 @@ def lib() -> ctypes.CDLL:
     L.kie_pending.argtypes = [VP]
     L.kie_pending.restype = ctypes.c_int32
     L.kie_get_info.argtypes = [VP, P(kie_info)]
+    L.kie_plan.argtypes = [P(kie_config), ctypes.c_int32, ctypes.c_int32, P(kie_plan_info),
+                           P(kie_seg_range), ctypes.c_int64]
     for f in ("kie_create", "kie_load_weights", "kie_prefill", "kie_decode", "kie_decode_static",
-              "kie_rewind", "kie_reset", "kie_destroy", "kie_get_info"):
+              "kie_rewind", "kie_reset", "kie_destroy", "kie_get_info", "kie_plan"):
         getattr(L, f).restype = ctypes.c_int
     _lib = L
     return L
@@ -100,6 +118,28 @@ def config_from(shape, max_ctx: int | None = None) -> kie_config:
                       ffn_expert=g("ffn_expert"), ffn_shared=g("ffn_shared"),
                       max_ctx=int(max_ctx if max_ctx is not None else shape.max_ctx),
                       rms_eps=float(shape.rms_eps), rope_theta=float(shape.rope_theta))
+
+
+def plan(shape, grid: int, stage_bytes: int, max_ctx: int | None = None):
+    """The weight-tape plan (kie_plan) for `grid` CTAs and ring stages of
+    `stage_bytes`: (info dict with per-kind tile shapes, ranges as a structured
+    numpy array [grid, ranges_per_cta] of (off, row0, nrows)). Host only."""
+    L = lib()
+    cfg = config_from(shape, max_ctx)
+    info = kie_plan_info()
+    st = L.kie_plan(ctypes.byref(cfg), int(grid), int(stage_bytes), ctypes.byref(info), None, 0)
+    if st != KIE_OK:
+        raise KieError(st, L.kie_last_error(None).decode())
+    n = grid * info.ranges_per_cta
+    buf = (kie_seg_range * n)()
+    st = L.kie_plan(ctypes.byref(cfg), int(grid), int(stage_bytes), ctypes.byref(info), buf, n)
+    if st != KIE_OK:
+        raise KieError(st, L.kie_last_error(None).decode())
+    dt = np.dtype([("off", np.int64), ("row0", np.int32), ("nrows", np.int32)])
+    ranges = np.frombuffer(bytes(buf), dtype=dt).reshape(grid, info.ranges_per_cta)
+    shapes = {k: dict(K=sh.K, g=sh.g, nk=sh.nk, kc=sh.kc) for k, sh in zip(SEG_KINDS, info.shapes)}
+    return dict(slots=info.slots, ranges_per_cta=info.ranges_per_cta, tape_bytes=info.tape_bytes,
+                shapes=shapes), ranges
 
 
 def _stream_ptr(stream=None) -> int:
