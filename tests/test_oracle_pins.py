@@ -390,3 +390,80 @@ def test_kv_cache_holds_fp16_rounded_values():
     for t in toks:
         m2.step(t, c2)
     assert not np.array_equal(c2["V"][:, :, :3, :], V)
+
+
+@pytest.mark.parametrize("hk", [2, 1], ids=["mha", "gqa2:1"])
+def test_rope_wiring_in_the_model_brute_force(hk):
+    # One layer whose q, k and v are known multiples of the normalised input:
+    # Wq = Wk = 3 I (per head), Wv = Wo = I, FFN output 0, lm_head = I, final
+    # gain 1. The expected logits are built with scalar loops: q and k of the
+    # token at position p are rotated by the angles of position p (pairs i,
+    # i + dh/2, angle p * theta^(-2i/dh)); v is not rotated; K (after the
+    # rotation) and V enter the cache rounded to fp16; causal softmax over
+    # j <= p with max subtraction. Large scores make the attention weights, and
+    # so the logits, depend on every rotation angle; the cache check fixes the
+    # absolute position at which k is rotated. A model that leaves k unrotated,
+    # rotates v, or rotates at position p + 1 fails here.
+    d, hq, dh, theta = 8, 2, 4, 10.0
+    s = S.Shape("t-rope", n_layers=1, d_model=d, n_heads=hq, n_kv_heads=hk, head_dim=dh, ffn=4,
+                vocab=11, max_ctx=8, rope_theta=theta)
+    w = S.make_weights(s, seed=13, cache=False)
+    w["layers.0.wq"][:] = 3 * np.eye(hq * dh, d, dtype=np.float16)
+    w["layers.0.wk"][:] = 3 * np.eye(hk * dh, d, dtype=np.float16)
+    w["layers.0.wv"][:] = np.eye(hk * dh, d, dtype=np.float16)
+    w["layers.0.wo"][:] = np.eye(d, hq * dh, dtype=np.float16)
+    w["layers.0.w_down"][:] = 0
+    w["final_norm"][:] = 1
+    w["lm_head"] = np.eye(11, d, dtype=np.float16)
+    toks = [5, 2, 9, 2, 7, 0]
+    T = len(toks)
+    g1 = [float(v) for v in w["layers.0.attn_norm"]]
+
+    def nrm(v, g):
+        r = math.sqrt(sum(a * a for a in v) / len(v) + s.rms_eps)
+        return [v[i] / r * g[i] for i in range(len(v))]
+
+    def rot(u, pos):  # one head's dh values
+        out = list(u)
+        for i in range(dh // 2):
+            phi = pos * theta ** (-2.0 * i / dh)
+            a, b = u[i], u[i + dh // 2]
+            out[i] = a * math.cos(phi) - b * math.sin(phi)
+            out[i + dh // 2] = a * math.sin(phi) + b * math.cos(phi)
+        return out
+
+    f16 = lambda v: float(np.float16(v))
+    xs = [[float(v) for v in w["embed"][t]] for t in toks]
+    xn = [nrm(x, g1) for x in xs]
+    # per position and KV head: cached K (rotated, fp16) and V (fp16)
+    Kc = [[[f16(v) for v in rot([3 * xn[j][g * dh + e] for e in range(dh)], j)] for g in range(hk)]
+          for j in range(T)]
+    Vc = [[[f16(xn[j][g * dh + e]) for e in range(dh)] for g in range(hk)] for j in range(T)]
+    want = []
+    for p in range(T):
+        o = []
+        for h in range(hq):
+            g = (h * hk) // hq
+            qh = rot([3 * xn[p][h * dh + e] for e in range(dh)], p)
+            sc = [sum(qh[e] * Kc[j][g][e] for e in range(dh)) / math.sqrt(dh) for j in range(p + 1)]
+            m = max(sc)
+            ex = [math.exp(v - m) for v in sc]
+            z = sum(ex)
+            o += [sum(ex[j] / z * Vc[j][g][e] for j in range(p + 1)) for e in range(dh)]
+        x2 = [xs[p][i] + o[i] for i in range(d)]
+        lg = nrm(x2, [1.0] * d) + [0.0] * 3
+        want.append(lg)
+    want = np.array(want)
+    # the attention weights are far from uniform, so the rotations matter
+    assert np.ptp(want[:, :d]) > 1.0
+
+    m = O.Decoder(s, w)
+    full = m.forward_sequence(toks)
+    assert np.allclose(full, want, rtol=0, atol=1e-12)
+    cache = m.new_cache(T)
+    for p in range(T):
+        assert np.allclose(m.step(toks[p], cache), want[p], rtol=0, atol=1e-12)
+    for j in range(T):
+        for g in range(hk):
+            assert list(cache["K"][0, g, j]) == Kc[j][g]
+            assert list(cache["V"][0, g, j]) == Vc[j][g]
