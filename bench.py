@@ -35,6 +35,8 @@ import sys
 import tempfile
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
@@ -213,6 +215,77 @@ def run_reference(args, shape):
     print(json.dumps(line), flush=True)
 
 
+PHASE_KINDS = ("qkv", "attention", "o_proj", "gate_up", "down", "lm_head")
+
+
+def summarize_phase_trace(t: np.ndarray, n_layers: int) -> dict:
+    """Per-token phase times from a trace-build record array t [grid, steps *
+    (5 L + 2), 4] (start, input ready, tiles done, epilogue done; the step
+    barrier last in each step as arrival, release, release, release).
+
+    Per CTA and step, each phase kind's input wait (start -> input ready),
+    tile time and epilogue time are summed over the layers; the figures are
+    medians over CTAs of the per-step mean. The step time is the interval
+    between consecutive barrier releases (median over CTAs); the wait share is
+    the phases' input waits plus the barrier wait over the step time."""
+    G, R, _ = t.shape
+    rps = 5 * n_layers + 2
+    steps = R // rps
+    t = t[:, :steps * rps].reshape(G, steps, rps, 4).astype(np.float64)
+    bar = t[:, :, rps - 1, :]
+    rel = np.median(bar[:, :, 1], axis=0)
+    step_us = float(np.diff(rel).mean() / 1000.0) if steps > 1 else float("nan")
+    out = {"steps": int(steps), "step_us": step_us, "per_token_us": {}}
+    total_wait = np.zeros((G, steps))
+    for k, name in enumerate(PHASE_KINDS):
+        idx = [n_layers * 5] if name == "lm_head" else [l * 5 + k for l in range(n_layers)]
+        rec = t[:, :, idx, :]
+        if not np.any(rec[..., 3] > 0):
+            continue
+        wait = (rec[..., 1] - rec[..., 0]).sum(axis=2)
+        tiles = (rec[..., 2] - rec[..., 1]).sum(axis=2)
+        epi = (rec[..., 3] - rec[..., 2]).sum(axis=2)
+        total_wait += wait
+        med = lambda a: float(np.median(a.mean(axis=1)) / 1000.0)
+        out["per_token_us"][name] = {"input_wait": med(wait), "tiles": med(tiles), "epilogue": med(epi)}
+    bw = bar[:, :, 1] - bar[:, :, 0]
+    out["per_token_us"]["step_barrier"] = {"wait": float(np.median(bw.mean(axis=1)) / 1000.0)}
+    if steps > 1:
+        span = float(np.median(np.diff(bar[:, :, 1], axis=1).sum(axis=1)))
+        out["flag_wait_share"] = float(np.median(total_wait[:, 1:].sum(axis=1)) / span)
+        out["barrier_wait_share"] = float(np.median(bw[:, 1:].sum(axis=1)) / span)
+    return out
+
+
+def phase_trace(shape, weights, prompt, device: int, m: int) -> dict:
+    """Run the trace build (libkie_trace.so) over the first and the last m
+    steps of the workload's decode and summarize both (see
+    summarize_phase_trace)."""
+    import torch
+    from transformer_decode_persistent_b200 import Engine
+    P, n = len(prompt), shape.decode_len
+    eng = Engine(shape, device=device, max_ctx=P + n, trace_build=True)
+    eng.load_weights(weights)
+    grid = eng.info()["grid"]
+    cap = m * (5 * shape.n_layers + 2)
+    res = {}
+    eng.prefill(prompt)
+    if n > m:
+        eng.decode(n - m)
+        tr = torch.zeros((grid, cap, 4), dtype=torch.int64, device=f"cuda:{device}")
+        eng.decode(m, trace=tr)
+        res["last"] = summarize_phase_trace(tr.cpu().numpy(), shape.n_layers)
+        res["last"]["positions"] = [P - 1 + n - m, P - 2 + n]
+        eng.reset()
+        eng.prefill(prompt)
+    tr = torch.zeros((grid, cap, 4), dtype=torch.int64, device=f"cuda:{device}")
+    eng.decode(m, trace=tr)
+    res["first"] = summarize_phase_trace(tr.cpu().numpy(), shape.n_layers)
+    res["first"]["positions"] = [P - 1, P - 2 + m]
+    eng.close()
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -224,7 +297,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--trace", action="store_true",
-                    help="also run traced decodes: step-barrier wait share, per-step time of the first and last 64 steps")
+                    help="also run the trace build over the first and last 64 steps: per-phase input wait, "
+                         "tile and epilogue time per token, flag-wait share")
     args = ap.parse_args()
 
     import synthetic as S
@@ -331,30 +405,7 @@ def main():
 
     stall = None
     if args.trace and rank == 0:
-        # globaltimer stamps of the step barrier (arrival, release) per CTA:
-        # the share of time CTAs wait in it, and the per-step time from one
-        # release to the next, over the first and the last 64 steps
-        m = min(n, 64)
-        cap = m * info["barriers_per_token"]
-
-        def traced(pos, tok):
-            tr = torch.zeros((info["grid"], cap, 2), dtype=torch.int64, device="cuda")
-            eng.rewind(pos, tok)
-            r = eng.decode(m, trace=tr)
-            return tr.cpu().numpy().astype(np.float64), r["tokens"]
-
-        stall = {}
-        if n > m:  # the last steps first: rewind only moves back from the current position
-            toks = out.cpu().numpy()
-            t2, _ = traced(P - 1 + n - m, int(toks[n - m - 1]))
-            rel2 = np.median(t2[:, :, 1], axis=0)
-            stall["step_us_last"] = float(np.diff(rel2).mean() / 1000.0)
-        t, _ = traced(P - 1, int(prompt[-1]))
-        span = t[:, :, 1].max() - t[:, :, 0].min()
-        stall["barrier_wait_share"] = float(((t[:, :, 1] - t[:, :, 0]).sum(axis=1) / span).mean())
-        rel = np.median(t[:, :, 1], axis=0)
-        stall["step_us_first"] = float(np.diff(rel).mean() / 1000.0)
-        stall["steps_averaged"] = m
+        stall = phase_trace(shape, weights, prompt, local, min(n, 64))
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:

@@ -57,7 +57,15 @@ typedef enum {
  * and ffn > 0; MoE models set ffn = 0 and the four expert fields.
  * Constraints: d_model, n_heads*head_dim, ffn, ffn_expert, ffn_shared multiples
  * of 8; head_dim 64 or 128; each KV head serves 1 to 4 query heads (query
- * head h reads KV head floor(h * n_kv_heads / n_heads)); max_ctx >= 1. */
+ * head h reads KV head floor(h * n_kv_heads / n_heads)); max_ctx >= 1.
+ * Capacity of one launch (one CTA per SM, S SMs): the rows of every matrix are
+ * split over the CTAs, and a CTA keeps at most 64 residual rows (d_model <=
+ * 64 S, checked by kie_create) and at most 1280 partial sums per phase (its
+ * rows of the matrix times the matrix's column blocks of 512 or 768 inputs).
+ * With S = 148 and d_model = 2560 (5 column blocks) that bounds the vocabulary
+ * at 37,888 and the gate/up width at 18,944 (2 ffn rows of 5 blocks each per
+ * unit). kie_load_weights and kie_plan reject a shape past these bounds with
+ * KIE_ERR_INVALID_ARG ("a CTA would hold N partial sums (max 1280)"). */
 typedef struct {
   int32_t n_layers, d_model, n_heads, n_kv_heads, head_dim, ffn, vocab;
   int32_t n_experts, top_k, ffn_expert, ffn_shared;
@@ -85,7 +93,9 @@ typedef struct {
 } kie_tensor;
 
 /* Optional per-call controls of kie_decode (pass NULL for defaults). Every
- * pointer may be host or device memory (detected per call), caller-owned. */
+ * pointer except trace_out may be host or device memory (detected per call),
+ * caller-owned; device memory must belong to the context's device
+ * (KIE_ERR_INVALID_ARG otherwise). */
 typedef struct {
   const int32_t* forced_tokens; /* [n]: token fed back after step i; -1 = argmax.
                                    Used for teacher forcing; NULL = free run.   */
@@ -94,8 +104,9 @@ typedef struct {
   uint32_t timeout_ms;          /* deadline of every device-side wait; 0 = 1000 ms    */
   int32_t fault_cta;            /* test hook: this CTA skips its arrival at grid      */
   int32_t fault_barrier;        /*   barrier number fault_barrier; -1 = off           */
-  uint64_t* trace_out;          /* device [grid][trace_cap][2] globaltimer stamps of
-                                   each grid barrier's arrival and release; NULL = off */
+  uint64_t* trace_out;          /* device memory of the context's device,
+                                   [grid][trace_cap][2] globaltimer stamps of each
+                                   grid barrier's arrival and release; NULL = off */
   int32_t trace_cap;            /* barriers recorded per CTA                          */
 } kie_decode_opts;
 
@@ -158,14 +169,16 @@ kie_status kie_decode(kie_ctx* ctx, int n_tokens, int32_t* out_tokens,
  * GPU that loads the library holds until the process exits. Models whose
  * scratch (8 bytes per flagged value: two residual copies, q/k/v, attention
  * output, FFN hidden; plus attention partials) exceeds it are rejected with KIE_ERR_INVALID_ARG
- * and a message giving both sizes. `out_tokens` must be device memory
- * ([n_tokens] int32, caller-owned); no logits, margins, forced tokens or trace.
+ * and a message giving both sizes. `out_tokens` must be device memory of
+ * the context's device ([n_tokens] int32, caller-owned); no logits, margins,
+ * forced tokens or trace.
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
  * capture. Every call on every context of a device shares the one array:
  * calls whose work overlaps on the GPU race and give wrong results; issue
- * them one after another. Errors: as kie_decode, plus INVALID_ARG for a host
- * `out_tokens` or a model whose scratch does not fit. */
+ * them one after another. Errors: as kie_decode, plus INVALID_ARG for an
+ * `out_tokens` that is not memory of the context's device, or a model whose
+ * scratch does not fit. */
 kie_status kie_decode_static(kie_ctx* ctx, int n_tokens, int32_t* out_tokens, void* stream);
 
 /* Truncate the sequence to its first `pos` committed positions (0 <= pos <=

@@ -206,7 +206,7 @@ class Decoder:
         self._w64 = {} if cache_f64 else None
         self.kv = fp16_round if kv_fp16 else f64
         # gap between the k-th and (k+1)-th router probability of every MoE
-        # decision taken by ``step`` (how close each routing was to a tie)
+        # decision taken (how close each routing was to a tie)
         self.route_gaps: list[float] = []
 
     def W(self, name: str) -> np.ndarray:
@@ -230,6 +230,10 @@ class Decoder:
                   self.W(p + "shared.w_down"))
         if np.ndim(xn) == 1:
             return moe_ffn(xn, self.W(p + "router"), experts, shared, s.top_k)
+        # diagnostic only: how close each row's routing came to a tie
+        for r in softmax(xn @ self.W(p + "router").T):
+            srt = np.sort(r)[::-1]
+            self.route_gaps.append(float(srt[s.top_k - 1] - srt[s.top_k]))
         return np.stack([moe_ffn(r, self.W(p + "router"), experts, shared, s.top_k)
                          for r in xn])
 

@@ -53,7 +53,7 @@ def make_engine(shape, weights, max_ctx=None, device=0):
 
 
 def forced_sequence_case(shape, seed: int, n: int, prompt_len: int | None = None,
-                         weights=None, engine=None):
+                         weights=None, engine=None, oracle=None):
     """Teacher forcing with a seeded continuation: the oracle computes every
     position in one full-sequence forward; the engine decodes n steps with the
     continuation forced. Returns (gpu_logits, oracle_logits, gpu_tokens)."""
@@ -61,7 +61,7 @@ def forced_sequence_case(shape, seed: int, n: int, prompt_len: int | None = None
     prompt = S.make_prompt(shape, seed, prompt_len)
     cont = S.make_tokens(shape, n, seed)
     P = len(prompt)
-    ref = O.Decoder(shape, w)
+    ref = oracle or O.Decoder(shape, w)
     ol = ref.forward_sequence(np.concatenate([prompt, cont[:n - 1]]))[P - 1:P - 1 + n]
     eng = engine or make_engine(shape, w, max_ctx=P + n)
     eng.reset()
@@ -98,3 +98,25 @@ def check_free_run(free_tokens, oracle_tokens, oracle_margins):
     assert np.array_equal(np.asarray(free_tokens[:k]), oracle_tokens[:k]), \
         f"free run diverges before step {k}"
     return k
+
+
+def free_run_case(shape, seed: int, n: int, prompt_len: int | None = None, weights=None,
+                  engine=None, oracle=None):
+    """The engine decodes n tokens free-running (greedy, one launch, logits
+    kept); the oracle then computes every step's logits from the same history
+    (prompt + the engine's own tokens) in one full-sequence forward. If the
+    engine's token equals the oracle's argmax at every step whose oracle margin
+    exceeds 0.05, the engine's free run is, by induction, the oracle's own
+    greedy run up to the first step with a smaller margin. Returns
+    (gpu_logits, oracle_logits, gpu_tokens, gpu_margins, oracle)."""
+    w = weights if weights is not None else S.make_weights(shape, seed)
+    prompt = S.make_prompt(shape, seed, prompt_len)
+    P = len(prompt)
+    eng = engine or make_engine(shape, w, max_ctx=P + n)
+    eng.reset()
+    eng.prefill(prompt)
+    r = eng.decode(n, logits=True, margins=True)
+    toks = np.asarray(r["tokens"]).astype(np.int64)
+    ref = oracle or O.Decoder(shape, w)
+    ol = ref.forward_sequence(np.concatenate([prompt, toks[:n - 1]]))[P - 1:P - 1 + n]
+    return r["logits"].cpu().numpy(), ol, toks, r["margins"].cpu().numpy(), ref

@@ -7,8 +7,9 @@ import numpy as np
 import pytest
 
 import synthetic as S
+import oracle as O
 from parity import (check_free_run, check_step_logits, check_tokens, forced_sequence_case,
-                    greedy_case, make_engine)
+                    free_run_case, greedy_case, make_engine)
 
 pytestmark = pytest.mark.gpu
 
@@ -156,3 +157,119 @@ def test_long_context_full_size_self_consistency():
     assert np.array_equal(a["logits"].cpu().numpy(), b["logits"].cpu().numpy())
     lg = a["logits"].cpu().numpy()
     assert np.isfinite(lg).all() and (np.std(lg, axis=1) > 0.1).all()
+
+
+def test_dense_2b_benchmarked_run():
+    # The run the benchmark times, in full: the 2.2B workload, prompt 256, 1024
+    # greedy tokens in one launch (positions 255-1278, attention split over up
+    # to 6 chunks per head). Every step's logits against the oracle on the
+    # same history; tokens exact at every confident step, so the free run is
+    # the oracle's greedy run up to its first step with margin <= 0.05.
+    s = S.DENSE_2B
+    gl, ol, gt, gm, _ = free_run_case(s, 0, s.decode_len)
+    check_step_logits(gl, ol, "2.2B 1024 steps")
+    check_tokens(gt, ol, "2.2B 1024 steps")
+    # the in-kernel margins are those of the kernel's own logits
+    srt = np.sort(gl, axis=-1)
+    assert np.array_equal(gm, srt[:, -1] - srt[:, -2])
+
+
+def test_long_context_reduced_oracle_parity():
+    # The long-context workload's weights and head layout (GQA 20:8 at d 2560)
+    # with the prompt cut to 2048 tokens and 32 greedy steps, as far as the
+    # oracle can follow.
+    s = S.LONG_2B_REDUCED
+    gl, ol, gt, _, _ = free_run_case(s, 0, s.decode_len)
+    check_step_logits(gl, ol, "2.2B GQA 20:8, 2K context")
+    check_tokens(gt, ol, "2.2B GQA 20:8, 2K context")
+
+
+def test_moe_full_size_64_steps():
+    # The MoE workload at full size: prompt 128, 64 greedy steps. A routing
+    # decision that the oracle takes within 1e-6 of a tie could go the other
+    # way in fp32; none may occur for the comparison to be meaningful.
+    s = S.MOE
+    gl, ol, gt, _, ref = free_run_case(s, 0, 64)
+    assert min(ref.route_gaps) > 1e-6, f"routing within {min(ref.route_gaps):.1e} of a tie"
+    check_step_logits(gl, ol, "moe 64 steps")
+    check_tokens(gt, ol, "moe 64 steps")
+
+
+@pytest.mark.parametrize("pair", [(7, 4001), (1200, 1201), (3000, 3)], ids=str)
+def test_planted_lm_head_tie_takes_the_lower_index(pair):
+    # Two identical LM-head rows that win every step: the kernel must report
+    # both logits bit-identical, choose the lower row index and a margin of
+    # exactly 0. The rows have one non-zero weight, so their logit is one
+    # rounded product whatever the summation order. Output and down
+    # projections are zero, so the final hidden state is the embedding of the
+    # (forced, constant) input token and the winning column is known.
+    s = S.TINY
+    w = S.make_weights(s, seed=21, cache=False)
+    for l in range(s.n_layers):
+        w[f"layers.{l}.wo"][:] = 0
+        w[f"layers.{l}.w_down"][:] = 0
+    t0 = 123
+    e = w["embed"][t0].astype(np.float64)
+    xn = e / np.sqrt(np.mean(e * e) + s.rms_eps) * w["final_norm"].astype(np.float64)
+    k = int(np.argmax(np.abs(xn)))
+    row = np.zeros(s.d_model, dtype=np.float16)
+    row[k] = np.float16(64.0 * np.sign(xn[k]))
+    for i in pair:
+        w["lm_head"][i] = row
+    eng = make_engine(s, w)
+    prompt = np.array([t0], dtype=np.int32)
+    n = 12
+    eng.prefill(prompt)
+    r = eng.decode(n, forced=np.full(n, t0, dtype=np.int32), logits=True, margins=True)
+    g = r["logits"].cpu().numpy()
+    lo, hi = min(pair), max(pair)
+    assert np.array_equal(g[:, lo], g[:, hi])
+    assert (np.argmax(g, axis=1) == lo).all()          # numpy also takes the first maximum
+    assert (np.asarray(r["tokens"]) == lo).all()
+    assert (r["margins"].cpu().numpy() == 0.0).all()
+    ol = O.Decoder(s, w).forward_sequence(np.full(n, t0))
+    check_step_logits(g, ol, "planted tie")
+    assert all(O.argmax_lowest(x) == lo for x in ol)
+
+
+def test_planted_router_tie_takes_the_lower_expert():
+    # Router rows: expert 6 = 2r, experts 2 and 5 = r (an exact tie), all
+    # others = -r, in every layer. With s = r . xn > 0 the top-2 are {6, 2}: the
+    # tie between 2 and 5 for the second slot goes to 2; with s < 0 the five
+    # others tie at the top and the two lowest, {0, 1}, win. Identical,
+    # negated and doubled rows give bit-identical, negated and doubled logits
+    # in any fixed summation order, so the kernel meets an exact tie; the
+    # experts' own weights differ, so taking the wrong one changes the logits.
+    s = MOE_SMALL
+    w = S.make_weights(s, seed=22, cache=False)
+    for l in range(s.n_layers):
+        R = w[f"layers.{l}.router"]
+        r = R[0].copy()
+        for e in range(s.n_experts):
+            R[e] = -r
+        R[2] = r
+        R[5] = r
+        R[6] = (2 * r.astype(np.float32)).astype(np.float16)
+    prompt = S.make_prompt(s, 22)
+    ref = O.Decoder(s, w)
+    ot, ol, om = ref.greedy(prompt, s.decode_len)
+    assert min(ref.route_gaps) == 0.0       # the ties really are met
+    eng = make_engine(s, w)
+    eng.prefill(prompt)
+    forced = eng.decode(s.decode_len, forced=ot.astype(np.int32), logits=True)
+    check_step_logits(forced["logits"].cpu().numpy(), ol, "router tie")
+    check_tokens(forced["tokens"], ol, "router tie")
+
+
+@pytest.mark.parametrize("which", ["small", "dense2b"])
+def test_fp16_cache_error_against_unrounded_definition(which):
+    # The kernel keeps K and V in fp16 (the workloads' cache); the oracle by
+    # default rounds them the same way. Against the unrounded fp64 definition
+    # the kernel must still meet the stated logit tolerances.
+    s = S.SMALL if which == "small" else S.DENSE_2B
+    w = S.make_weights(s, seed=0)
+    n = 24 if which == "small" else 6
+    ref = O.Decoder(s, w, kv_fp16=False)
+    gl, ol, gt, _ = forced_sequence_case(s, 0, n, weights=w, oracle=ref)
+    check_step_logits(gl, ol, f"{which} vs unrounded cache")
+    check_tokens(gt, ol, f"{which} vs unrounded cache")

@@ -1,4 +1,9 @@
-"""Build libkie.so in-tree with nvcc for sm_100a (B200).
+"""Build the decode library in-tree with nvcc for sm_100a (B200).
+
+Two libraries from the same sources: libkie.so (the product) and
+libkie_trace.so (compiled with KIE_TRACE: the kernel also stamps the start,
+input-ready, tiles-done and epilogue-done times of every phase into the
+caller's trace buffer; used for measurement only).
 
 Usage: python -m transformer_decode_persistent_b200.build [--verbose]
 """
@@ -12,6 +17,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libkie.so")
+LIB_TRACE = os.path.join(HERE, "libkie_trace.so")
 SOURCES = ["monokernel.cu", "kie_host.cu"]
 HEADERS = ["kie_internal.h", os.path.join("..", "..", "include", "kie.h")]
 
@@ -27,20 +33,19 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, s) for s in SOURCES + HEADERS] + [os.path.abspath(__file__)]
     return any(os.path.getmtime(p) > t for p in deps if os.path.exists(p))
 
 
-def build(verbose: bool = False, force: bool = False, ptxas_info: bool = False) -> str:
-    """Compile the CUDA sources into libkie.so next to this file; returns its path."""
-    if not force and not _stale():
-        return LIB
-    tmp = LIB + f".{os.getpid()}.tmp"
-    cmd = [nvcc(), *ARCH, *FLAGS, "-shared", "-o", tmp,
+def _build_one(lib: str, defines, verbose: bool, force: bool, ptxas_info: bool) -> str:
+    if not force and not _stale(lib):
+        return lib
+    tmp = lib + f".{os.getpid()}.tmp"
+    cmd = [nvcc(), *ARCH, *FLAGS, *defines, "-shared", "-o", tmp,
            *[os.path.join(CSRC, s) for s in SOURCES]]
     if ptxas_info:
         cmd.insert(1, "-Xptxas=-v")
@@ -49,10 +54,18 @@ def build(verbose: bool = False, force: bool = False, ptxas_info: bool = False) 
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
-        raise RuntimeError("nvcc failed building libkie.so")
+        raise RuntimeError(f"nvcc failed building {os.path.basename(lib)}")
     if verbose or ptxas_info:
         sys.stdout.write(r.stdout + r.stderr)
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+    return lib
+
+
+def build(verbose: bool = False, force: bool = False, ptxas_info: bool = False) -> str:
+    """Compile the CUDA sources into libkie.so and libkie_trace.so next to this
+    file; returns the product library's path."""
+    _build_one(LIB, [], verbose, force, ptxas_info)
+    _build_one(LIB_TRACE, ["-DKIE_TRACE"], verbose, force, False)
     return LIB
 
 

@@ -121,13 +121,25 @@ void dfree(kie_ctx* c, void* p) {
   cudaFree(p);
 }
 
-bool is_device_ptr(const void* p) {
+// CUDA device owning `p` (device or managed memory), or -1 for host memory.
+int ptr_device(const void* p) {
   cudaPointerAttributes a{};
   if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
     cudaGetLastError();
-    return false;
+    return -1;
   }
-  return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+  return (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) ? a.device : -1;
+}
+
+bool is_device_ptr(const void* p) { return ptr_device(p) >= 0; }
+
+// INVALID_ARG if `p` is device memory of a device other than the context's.
+kie_status check_own_device(kie_ctx* c, const void* p, const char* what) {
+  const int dev = p ? ptr_device(p) : -1;
+  if (dev >= 0 && dev != c->device)
+    return fail(c, KIE_ERR_INVALID_ARG, "%s is memory of device %d; the context is on device %d", what, dev,
+                c->device);
+  return KIE_OK;
 }
 
 // Tile shape for a segment kind: rows per tile g and column chunks nk. Prefer
@@ -662,8 +674,9 @@ kie_status kie_load_weights(kie_ctx* c, const kie_tensor* tensors, int n, void* 
       return fail(c, KIE_ERR_INVALID_ARG, "tensor '%s' has shape [%lld, %lld], expected [%lld, %lld]",
                   t.name, (long long)t.shape[0], (long long)t.shape[1], (long long)it->second.first,
                   (long long)it->second.second);
-    if (t.on_device && !is_device_ptr(t.data))
-      return fail(c, KIE_ERR_INVALID_ARG, "tensor '%s' marked on_device but is not device memory", t.name);
+    if (t.on_device && ptr_device(t.data) != c->device)
+      return fail(c, KIE_ERR_INVALID_ARG, "tensor '%s' marked on_device but is not memory of device %d", t.name,
+                  c->device);
     if (t.on_device && (reinterpret_cast<uintptr_t>(t.data) & 15))
       return fail(c, KIE_ERR_INVALID_ARG, "device tensor '%s' is not 16-byte aligned", t.name);
     got[t.name] = Tensor{t.data, r, cc, t.on_device != 0};
@@ -879,7 +892,11 @@ struct Run {
   int trace_cap;
 };
 
-kie_status launch(kie_ctx* c, const Run& r, cudaStream_t st) {
+// The kernel's parameter block for run `r`, with the per-launch scratch (the
+// region cleared before every launch: control block, arrival counters and
+// flagged words) at `sync_base` and the attention partials at `apart`. Both
+// entry points that launch the kernel build their parameters here.
+Params make_params(const kie_ctx* c, const Run& r, unsigned char* sync_base, float* apart) {
   const kie_config& k = c->cfg;
   Params P{};
   P.L = k.n_layers; P.d = k.d_model; P.hq = k.n_heads; P.hk = k.n_kv_heads; P.dh = k.head_dim;
@@ -892,8 +909,8 @@ kie_status launch(kie_ctx* c, const Run& r, cudaStream_t st) {
   P.embed = c->embed; P.attn_norm = c->attn_norm; P.mlp_norm = c->mlp_norm;
   P.final_norm = c->final_norm; P.router = c->router;
   P.kcache = c->kcache; P.vcache = c->vcache; P.rope = c->rope;
-  P.apart = c->apart;
-  set_sync_params(P, c->syncblk, sync_layout(k, c->grid, c->hbuf));
+  P.apart = apart;
+  set_sync_params(P, sync_base, sync_layout(k, c->grid, c->hbuf));
   P.max_chunks = c->max_chunks;
   P.pos0 = c->pos; P.n_steps = r.n_steps; P.first_token = r.first_token; P.lm_from_step = r.lm_from_step;
   P.forced = r.forced; P.out_tokens = r.out; P.logits_out = r.logits; P.margins_out = r.margins;
@@ -903,8 +920,17 @@ kie_status launch(kie_ctx* c, const Run& r, cudaStream_t st) {
   P.n_stages = c->n_stages; P.stage_bytes = c->stage_bytes; P.vec_floats = c->vec_floats;
   P.xplane = c->xplane;
   P.gbuf_off = c->gbuf_off;
+  return P;
+}
 
-  CUDA_TRY(c, cudaMemsetAsync(c->syncblk, 0, c->syncblk_bytes, st));
+// Clear the per-launch scratch at `sync_base` (`sync_bytes`), launch the
+// kernel for run `r`, wait for it and read its error record. On success the
+// pending token becomes the kernel's last one (position bookkeeping is the
+// caller's).
+kie_status launch_on(kie_ctx* c, const Run& r, unsigned char* sync_base, size_t sync_bytes, float* apart,
+                     cudaStream_t st) {
+  Params P = make_params(c, r, sync_base, apart);
+  CUDA_TRY(c, cudaMemsetAsync(sync_base, 0, sync_bytes, st));
   void* args[] = {&P};
   cudaError_t e = cudaLaunchCooperativeKernel(kernel_entry(), dim3(c->grid), dim3(kThreads), args,
                                               (size_t)c->smem, st);
@@ -919,7 +945,7 @@ kie_status launch(kie_ctx* c, const Run& r, cudaStream_t st) {
     return fail(c, KIE_ERR_CUDA, "decode kernel failed: %s", cudaGetErrorString(e));
   }
   Ctrl ctl{};
-  CUDA_TRY(c, cudaMemcpy(&ctl, c->syncblk, sizeof(Ctrl), cudaMemcpyDeviceToHost));
+  CUDA_TRY(c, cudaMemcpy(&ctl, sync_base, sizeof(Ctrl), cudaMemcpyDeviceToHost));
   if (ctl.err) {
     c->poisoned = true;
     static const char* where[] = {"?", "grid barrier", "ring stage (full)", "ring stage (empty)",
@@ -931,6 +957,11 @@ kie_status launch(kie_ctx* c, const Run& r, cudaStream_t st) {
   }
   c->pending = ctl.final_token;
   return KIE_OK;
+}
+
+// A launch with the context's own scratch.
+kie_status launch(kie_ctx* c, const Run& r, cudaStream_t st) {
+  return launch_on(c, r, c->syncblk, c->syncblk_bytes, c->apart, st);
 }
 
 }  // namespace
@@ -995,6 +1026,16 @@ kie_status kie_decode(kie_ctx* c, int n, int32_t* out_tokens, const kie_decode_o
   o.fault_barrier = -1;
   if (opts) o = *opts;
   if (o.trace_out && o.trace_cap <= 0) return fail(c, KIE_ERR_INVALID_ARG, "trace_cap must be > 0");
+  if (o.trace_out && ptr_device(o.trace_out) != c->device)
+    return fail(c, KIE_ERR_INVALID_ARG, "trace_out must be memory of device %d", c->device);
+  {
+    kie_status ps;
+    if ((ps = check_own_device(c, out_tokens, "out_tokens")) ||
+        (ps = check_own_device(c, o.forced_tokens, "forced_tokens")) ||
+        (ps = check_own_device(c, o.logits_out, "logits_out")) ||
+        (ps = check_own_device(c, o.margins_out, "margins_out")))
+      return ps;
+  }
   cudaSetDevice(c->device);
   cudaStream_t st = (cudaStream_t)stream;
   const int V = c->cfg.vocab;
@@ -1109,8 +1150,8 @@ extern "C" kie_status kie_decode_static(kie_ctx* c, int n, int32_t* out_tokens, 
   if (c->device < 0 || c->device >= kMaxDevices) return fail(c, KIE_ERR_INVALID_ARG, "device %d out of range", c->device);
   if (n < 0) return fail(c, KIE_ERR_INVALID_ARG, "negative token count");
   if (n == 0) return KIE_OK;
-  if (!out_tokens || !is_device_ptr(out_tokens))
-    return fail(c, KIE_ERR_INVALID_ARG, "out_tokens must be device memory");
+  if (!out_tokens || ptr_device(out_tokens) != c->device)
+    return fail(c, KIE_ERR_INVALID_ARG, "out_tokens must be memory of device %d", c->device);
   if (c->pending < 0) return fail(c, KIE_ERR_STATE, "no pending token: prefill first");
   if ((int64_t)c->pos + n > c->cfg.max_ctx)
     return fail(c, KIE_ERR_CONTEXT_FULL, "position %d + %d tokens exceeds max_ctx %d", c->pos, n, c->cfg.max_ctx);
@@ -1131,53 +1172,12 @@ extern "C" kie_status kie_decode_static(kie_ctx* c, int n, int32_t* out_tokens, 
     base = g_static_ptr[c->device];
   }
   cudaStream_t st = (cudaStream_t)stream;
-  const kie_config& k = c->cfg;
-  Params P{};
-  P.L = k.n_layers; P.d = k.d_model; P.hq = k.n_heads; P.hk = k.n_kv_heads; P.dh = k.head_dim;
-  P.ff = k.ffn; P.V = k.vocab; P.E = k.n_experts; P.top_k = k.top_k; P.ffe = k.ffn_expert;
-  P.ffs = k.ffn_shared; P.max_ctx = k.max_ctx; P.eps = k.rms_eps;
-  P.qkv_rows = (k.n_heads + 2 * k.n_kv_heads) * k.head_dim;
-  P.slots = c->slots;
-  P.tape = c->tape; P.desc = c->desc;
-  for (int i = 0; i < SK_COUNT; ++i) P.shp[i] = c->shp[i];
-  P.embed = c->embed; P.attn_norm = c->attn_norm; P.mlp_norm = c->mlp_norm;
-  P.final_norm = c->final_norm; P.router = c->router;
-  P.kcache = c->kcache; P.vcache = c->vcache; P.rope = c->rope;
-  P.apart = reinterpret_cast<float*>(base + lay.apart);
-  set_sync_params(P, base + lay.sync, sync_layout(k, c->grid, c->hbuf));
-  P.max_chunks = c->max_chunks;
-  P.pos0 = c->pos; P.n_steps = n; P.first_token = c->pending; P.lm_from_step = 0;
-  P.forced = nullptr; P.out_tokens = out_tokens; P.logits_out = nullptr; P.margins_out = nullptr;
-  P.timeout_ns = 1000ull * 1000000ull;
-  P.fault_cta = -1; P.fault_barrier = -1;
-  P.trace = nullptr; P.trace_cap = 0;
-  P.n_stages = c->n_stages; P.stage_bytes = c->stage_bytes; P.vec_floats = c->vec_floats;
-  P.xplane = c->xplane;
-  P.gbuf_off = c->gbuf_off;
   // the array keeps the previous call's contents: the barrier counter, the
   // abort flag, the attention arrival counters and the flagged words' epochs
-  // must start at zero
-  CUDA_TRY(c, cudaMemsetAsync(base + lay.sync, 0, lay.sync_bytes, st));
-  void* args[] = {&P};
-  cudaError_t e = cudaLaunchCooperativeKernel(kernel_entry(), dim3(c->grid), dim3(kThreads), args, (size_t)c->smem, st);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return fail(c, KIE_ERR_CUDA, "cooperative launch failed: %s", cudaGetErrorString(e));
-  }
-  c->launches++;
-  e = cudaStreamSynchronize(st);
-  if (e != cudaSuccess) {
-    c->poisoned = true;
-    return fail(c, KIE_ERR_CUDA, "decode kernel failed: %s", cudaGetErrorString(e));
-  }
-  Ctrl ctl{};
-  CUDA_TRY(c, cudaMemcpy(&ctl, base + lay.sync, sizeof(Ctrl), cudaMemcpyDeviceToHost));
-  if (ctl.err) {
-    c->poisoned = true;
-    return fail(c, (kie_status)ctl.err, "device %s (cta %d, step %d, where %d); context poisoned",
-                ctl.err == KIE_ERR_TIMEOUT ? "timeout" : "check failed", ctl.err_cta, ctl.err_step, ctl.err_where);
-  }
-  c->pending = ctl.final_token;
+  // must start at zero, which launch_on's clear of the sync region ensures
+  const Run r{c->pending, n, 0, nullptr, out_tokens, nullptr, nullptr, 0, -1, -1, nullptr, 0};
+  kie_status s = launch_on(c, r, base + lay.sync, lay.sync_bytes, reinterpret_cast<float*>(base + lay.apart), st);
+  if (s != KIE_OK) return s;
   c->pos += n;
   return KIE_OK;
 }

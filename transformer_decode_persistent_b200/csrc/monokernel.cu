@@ -460,6 +460,10 @@ struct Producer {
     const int nu = attn_units_of(ap, blockIdx.x, G);
     const int per_unit = ap.nsb * kAttnTilesPerRound;
     const int ntiles = nu * per_unit;
+    // The cache rows were written with generic stores by other CTAs in earlier
+    // steps (ordered before this point by the step barrier and the ring's
+    // mbarriers); order them before this lane's bulk (async-proxy) reads.
+    if (ntiles > 0) asm volatile("fence.proxy.async.global;" ::: "memory");
     for (int i = (int)((lane + ns - (int)(t % ns)) % ns); i < ntiles; i += ns) {
       const int uo = i / per_unit, r = i - uo * per_unit;
       const int b = r / kAttnTilesPerRound, ti = r - b * kAttnTilesPerRound;
@@ -657,6 +661,24 @@ struct Consumer {
 
   __device__ __forceinline__ int ap_nchk(int pos) const { return attn_plan(pos, P.hk, gridDim.x).nchk; }
 
+  // Phase trace (KIE_TRACE builds): per CTA and step, one record of four
+  // %globaltimer stamps per phase -- phase start (before its input wait),
+  // input ready, tiles (or attention) done, epilogue done -- and a last record
+  // for the step barrier (arrival, then release three times). Thread 0 writes
+  // the stamps; it passes every consumer barrier, so they are CTA-wide times.
+  __device__ __forceinline__ int trace_recs_per_step() const { return 5 * P.L + 2; }
+  __device__ __forceinline__ void tstamp(int ph, int i) {
+#ifdef KIE_TRACE
+    if (P.trace && tid == 0) {
+      const int rec = step * trace_recs_per_step() + ph;
+      if (rec < P.trace_cap) P.trace[((size_t)blockIdx.x * P.trace_cap + rec) * 4 + i] = gtimer();
+    }
+#else
+    (void)ph;
+    (void)i;
+#endif
+  }
+
   __device__ __forceinline__ unsigned epoch(int l) const { return 1u + (unsigned)step * (unsigned)(P.L + 1) + (unsigned)l; }
 
   // Four flagged words at p (16-byte aligned) once they all carry epoch ep.
@@ -842,11 +864,25 @@ struct Consumer {
         }
         asm volatile("fence.acq_rel.gpu;" ::: "memory");  // acquire the other CTAs' writes
       }
+#ifdef KIE_TRACE
+      if (P.trace) {
+        const int rec = step * trace_recs_per_step() + trace_recs_per_step() - 1;
+        if (rec < P.trace_cap) {
+          unsigned long long* tr = P.trace + ((size_t)blockIdx.x * P.trace_cap + rec) * 4;
+          const unsigned long long tb = gtimer();
+          tr[0] = ta;
+          tr[1] = tb;
+          tr[2] = tb;
+          tr[3] = tb;
+        }
+      }
+#else
       if (P.trace && (int)k < P.trace_cap) {
         unsigned long long* tr = P.trace + ((size_t)blockIdx.x * P.trace_cap + k) * 2;
         tr[0] = ta;
         tr[1] = gtimer();
       }
+#endif
       sc->abort = ab;
     }
     return !cbar_any(sc->abort != 0);
@@ -1286,6 +1322,7 @@ struct Consumer {
       for (int ph = 0; ph < nph; ++ph) {
         const int l = ph / 5;
         const int kind = (l == P.L) ? PH_LM : ph - l * 5;
+        tstamp(ph, 0);
         // ---- 1. input vector
         switch (kind) {
           case PH_QKV:
@@ -1319,6 +1356,7 @@ struct Consumer {
           default:
             break;
         }
+        tstamp(ph, 1);
         // ---- 2. tiles
         if (kind == PH_ATTN) {
           attention_dispatch(l, pos);
@@ -1353,6 +1391,7 @@ struct Consumer {
           }
         }
         cbar();
+        tstamp(ph, 2);
         // ---- 3. epilogue
         switch (kind) {
           case PH_QKV:
@@ -1381,6 +1420,7 @@ struct Consumer {
             break;
         }
         if (cbar_any(sc->abort != 0)) return;
+        tstamp(ph, 3);
       }
       int next;
       if (lm) {

@@ -14,6 +14,8 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkie.so")
+# the same library compiled with KIE_TRACE (per-phase timestamps; measurement only)
+LIB_TRACE_PATH = os.path.join(_HERE, "libkie_trace.so")
 
 KIE_OK = 0
 STATUS = {0: "KIE_OK", -1: "KIE_ERR_INVALID_ARG", -2: "KIE_ERR_STATE", -3: "KIE_ERR_CONTEXT_FULL",
@@ -72,18 +74,19 @@ class kie_plan_info(ctypes.Structure):
 SEG_KINDS = ("qkv", "o", "gate_up", "down", "shared_gate_up", "expert_gate_up", "shared_down",
              "expert_down", "lm_head")
 
-_lib = None
+_libs = {}
 
 
-def lib() -> ctypes.CDLL:
-    """Load libkie.so (built in-tree); raises if it has not been built."""
-    global _lib
-    if _lib is not None:
-        return _lib
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with "
+def lib(trace: bool = False) -> ctypes.CDLL:
+    """Load libkie.so (or, with ``trace``, libkie_trace.so), built in-tree;
+    raises if it has not been built."""
+    if trace in _libs:
+        return _libs[trace]
+    path = LIB_TRACE_PATH if trace else LIB_PATH
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
                           "`python -m transformer_decode_persistent_b200.build`")
-    L = ctypes.CDLL(LIB_PATH)
+    L = ctypes.CDLL(path)
     P, I, VP = ctypes.POINTER, ctypes.c_int, ctypes.c_void_p
     L.kie_create.argtypes = [P(kie_config), I, P(VP)]
     L.kie_load_weights.argtypes = [VP, P(kie_tensor), I, VP]
@@ -105,7 +108,7 @@ def lib() -> ctypes.CDLL:
     for f in ("kie_create", "kie_load_weights", "kie_prefill", "kie_decode", "kie_decode_static",
               "kie_rewind", "kie_reset", "kie_destroy", "kie_get_info", "kie_plan"):
         getattr(L, f).restype = ctypes.c_int
-    _lib = L
+    _libs[trace] = L
     return L
 
 
@@ -142,6 +145,27 @@ def plan(shape, grid: int, stage_bytes: int, max_ctx: int | None = None):
                 shapes=shapes), ranges
 
 
+def _check_out(out, n: int, device: int, need_cuda: bool = False):
+    """Raise unless ``out`` can take n int32 tokens: a contiguous int32 tensor
+    (CUDA on ``device``, or host) or a contiguous int32 numpy array."""
+    import torch
+    if isinstance(out, torch.Tensor):
+        if out.dtype != torch.int32 or not out.is_contiguous() or out.numel() < n:
+            raise ValueError(f"out must be a contiguous int32 tensor of >= {n} elements, got "
+                             f"{out.dtype} {tuple(out.shape)}")
+        if out.is_cuda and out.device.index != device:
+            raise ValueError(f"out is on {out.device}, the engine on cuda:{device}")
+        if need_cuda and not out.is_cuda:
+            raise ValueError("out must be a CUDA tensor")
+    else:
+        if need_cuda:
+            raise ValueError("out must be a CUDA tensor")
+        a = out
+        if not isinstance(a, np.ndarray) or a.dtype != np.int32 or not a.flags["C_CONTIGUOUS"] \
+                or a.size < n:
+            raise ValueError(f"out must be a contiguous int32 array of >= {n} elements")
+
+
 def _stream_ptr(stream=None) -> int:
     import torch
     s = stream if stream is not None else torch.cuda.current_stream()
@@ -151,9 +175,12 @@ def _stream_ptr(stream=None) -> int:
 class Engine:
     """One batch-1 decode context on one GPU (a thin wrapper over kie_ctx)."""
 
-    def __init__(self, shape, device: int = 0, max_ctx: int | None = None):
+    def __init__(self, shape, device: int = 0, max_ctx: int | None = None, trace_build: bool = False):
+        """``trace_build`` loads libkie_trace.so, whose decode also writes one
+        record of four phase timestamps per phase (see ``decode(trace=...)``)."""
         import torch
-        self.L = lib()
+        self.trace_build = trace_build
+        self.L = lib(trace_build)
         self.device = device
         self.cfg = config_from(shape, max_ctx)
         torch.cuda.init()
@@ -227,7 +254,10 @@ class Engine:
         and 'logits' ([n, V] float32 CUDA tensor) / 'margins' ([n] float32 CUDA
         tensor) when requested. ``out`` may be a CUDA int32 tensor or a host
         (pinned) int32 tensor / numpy array. ``trace`` is a CUDA int64 tensor
-        [grid, cap, 2] for barrier timestamps.
+        [grid, cap, 2] for the step barrier's arrival and release times, or,
+        on a trace-build engine, [grid, cap, 4] with one record per phase
+        (start, input ready, tiles done, epilogue done; records step * (5 L +
+        2) + phase, the step barrier last).
         """
         import torch
         o = kie_decode_opts(fault_cta=-1, fault_barrier=-1, timeout_ms=int(timeout_ms))
@@ -249,6 +279,13 @@ class Engine:
         if fault is not None:
             o.fault_cta, o.fault_barrier = int(fault[0]), int(fault[1])
         if trace is not None:
+            grid = self.info()["grid"]
+            if (not isinstance(trace, torch.Tensor) or trace.dtype != torch.int64 or not trace.is_cuda
+                    or trace.device.index != self.device or trace.dim() != 3
+                    or trace.shape[0] != grid or trace.shape[2] != self.trace_words
+                    or not trace.is_contiguous()):
+                raise ValueError(f"trace must be a contiguous int64 CUDA tensor "
+                                 f"[{grid}, cap, {self.trace_words}] on cuda:{self.device}")
             o.trace_out = trace.data_ptr()
             o.trace_cap = int(trace.shape[1])
         if out is None:
@@ -256,9 +293,11 @@ class Engine:
             optr = out_arr.ctypes.data
             res["tokens"] = out_arr
         elif isinstance(out, torch.Tensor):
+            _check_out(out, n, self.device)
             optr = out.data_ptr()
             res["tokens"] = out
         else:
+            _check_out(out, n, self.device)
             optr = out.ctypes.data
             res["tokens"] = out
         with torch.cuda.device(self.device):
@@ -270,6 +309,7 @@ class Engine:
         """kie_decode_static: n greedy tokens into ``out`` (a CUDA int32 tensor),
         with the kernel's scratch in the library's static device array."""
         import torch
+        _check_out(out, n, self.device, need_cuda=True)
         with torch.cuda.device(self.device):
             self._check(self.L.kie_decode_static(self.h, int(n), ctypes.c_void_p(out.data_ptr()),
                                                  ctypes.c_void_p(_stream_ptr(stream))))
@@ -280,6 +320,11 @@ class Engine:
 
     def rewind(self, pos: int, pending: int):
         self._check(self.L.kie_rewind(self.h, int(pos), int(pending)))
+
+    @property
+    def trace_words(self) -> int:
+        """Stamps per trace record: 4 in the trace build, 2 in the product."""
+        return 4 if self.trace_build else 2
 
     @property
     def position(self) -> int:
