@@ -205,8 +205,10 @@ class Decoder:
         self.w16 = weights
         self._w64 = {} if cache_f64 else None
         self.kv = fp16_round if kv_fp16 else f64
-        # gap between the k-th and (k+1)-th router probability of every MoE
-        # decision taken (how close each routing was to a tie)
+        # gap between the k-th and (k+1)-th largest router logit of every MoE
+        # decision taken (how close each routing was to a tie; diagnostic
+        # only). ``step`` appends one per layer; ``forward_sequence`` one per
+        # row for each layer in turn (layer-major).
         self.route_gaps: list[float] = []
 
     def W(self, name: str) -> np.ndarray:
@@ -231,7 +233,7 @@ class Decoder:
         if np.ndim(xn) == 1:
             return moe_ffn(xn, self.W(p + "router"), experts, shared, s.top_k)
         # diagnostic only: how close each row's routing came to a tie
-        for r in softmax(xn @ self.W(p + "router").T):
+        for r in xn @ self.W(p + "router").T:
             srt = np.sort(r)[::-1]
             self.route_gaps.append(float(srt[s.top_k - 1] - srt[s.top_k]))
         return np.stack([moe_ffn(r, self.W(p + "router"), experts, shared, s.top_k)
@@ -240,9 +242,10 @@ class Decoder:
     def _moe_ffn_lazy(self, l: int, xn):
         """One token's MoE FFN, widening only the experts it chooses."""
         s, p = self.s, f"layers.{l}."
-        r = softmax(xn @ self.W(p + "router").T)
+        logit = xn @ self.W(p + "router").T
+        r = softmax(logit)
         chosen = topk_lowest(r, s.top_k)
-        srt = np.sort(r)[::-1]
+        srt = np.sort(logit)[::-1]
         self.route_gaps.append(float(srt[s.top_k - 1] - srt[s.top_k]))
         wsum = sum(r[e] for e in chosen)
         y = swiglu_ffn(xn, self.W(p + "shared.w_gate"), self.W(p + "shared.w_up"),
