@@ -138,9 +138,12 @@ def test_gqa_long_context_multi_round_attention():
 def test_long_context_full_size_self_consistency():
     # The long-context workload at full size (32768-token prompt, GQA 20:8, fp16
     # KV cache of 3.5 GB). The oracle cannot run a 32K-token 2.2B prefix, so the
-    # check is a property: re-forwarding the last prompt tokens in decode mode
-    # (teacher-forced) after rewinding reproduces the same cache and therefore
-    # bit-identical logits and tokens, and repeated runs are deterministic.
+    # checks are properties. (a) Re-forwarding the last prompt tokens through
+    # the prompt path after a rewind rewrites the same cache entries, so the
+    # following logits and tokens are bit-identical (the prompt path's results
+    # do not depend on how the prompt is cut into calls or chunks). (b)
+    # Re-forwarding them through the decode kernel instead (teacher-forced)
+    # gives logits within the parity tolerance of the prompt path's.
     s = S.LONG_2B
     w = S.make_weights(s, seed=0)
     prompt = S.make_prompt(s, 0)
@@ -150,13 +153,57 @@ def test_long_context_full_size_self_consistency():
     a = eng.decode(16, logits=True)
     k = 8
     eng.rewind(P - 1 - k, int(prompt[P - 1 - k]))
-    f = eng.decode(k, forced=prompt[P - k:].astype(np.int32))
+    eng.prefill(prompt[P - k:])
     assert eng.position == P - 1 and eng.pending == int(prompt[-1])
     b = eng.decode(16, logits=True)
     assert np.array_equal(a["tokens"], b["tokens"])
     assert np.array_equal(a["logits"].cpu().numpy(), b["logits"].cpu().numpy())
+    eng.rewind(P - 1 - k, int(prompt[P - 1 - k]))
+    eng.decode(k, forced=prompt[P - k:].astype(np.int32))
+    assert eng.position == P - 1 and eng.pending == int(prompt[-1])
+    c = eng.decode(16, logits=True)
+    check_step_logits(c["logits"].cpu().numpy(), a["logits"].cpu().numpy().astype(np.float64),
+                      "decode-path re-forward vs prompt path")
     lg = a["logits"].cpu().numpy()
     assert np.isfinite(lg).all() and (np.std(lg, axis=1) > 0.1).all()
+
+
+def test_prompt_path_matches_decode_path_and_oracle():
+    # The tensor-core prompt path and the decode kernel run teacher-forced over
+    # the same prompt fill caches whose next 16 steps agree with each other and
+    # with the oracle under the parity criteria.
+    s = S.SMALL
+    w = S.make_weights(s, seed=0)
+    prompt = S.make_prompt(s, 0)
+    P = len(prompt)
+    eng = make_engine(s, w, max_ctx=P + 16)
+    eng.prefill(prompt)
+    a = eng.decode(16, logits=True, forced=S.make_tokens(s, 16, 9))
+    eng.reset()
+    eng.prefill(prompt[:1])
+    eng.decode(P - 1, forced=prompt[1:].astype(np.int32))
+    assert eng.position == P - 1 and eng.pending == int(prompt[-1])
+    b = eng.decode(16, logits=True, forced=S.make_tokens(s, 16, 9))
+    ga, gb = a["logits"].cpu().numpy(), b["logits"].cpu().numpy()
+    check_step_logits(ga, gb.astype(np.float64), "prompt path vs decode path")
+    cont = S.make_tokens(s, 16, 9)
+    ol = O.Decoder(s, w).forward_sequence(np.concatenate([prompt, cont[:15]]))[P - 1:]
+    check_step_logits(ga, ol, "prompt path vs oracle")
+    check_tokens(a["tokens"], ol, "prompt path vs oracle")
+
+
+RAGGED_LONG = S.Shape("ragged-long", n_layers=2, d_model=136, n_heads=2, n_kv_heads=1, head_dim=64,
+                      ffn=200, vocab=1001, prompt_len=300, decode_len=12, max_ctx=312)
+
+
+def test_prompt_path_ragged_tiles():
+    # widths that fill no tensor-core tile (d 136, q/k/v rows 256, gate/up rows
+    # 400, K 136 and 200) and a 300-token prompt over three 128-token tiles
+    s = RAGGED_LONG
+    w = S.make_weights(s, seed=6, cache=False)
+    gl, ol, gt, _ = forced_sequence_case(s, 6, s.decode_len, weights=w)
+    check_step_logits(gl, ol, "ragged prompt path")
+    check_tokens(gt, ol, "ragged prompt path")
 
 
 def test_dense_2b_benchmarked_run():

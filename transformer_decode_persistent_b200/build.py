@@ -18,8 +18,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libkie.so")
 LIB_TRACE = os.path.join(HERE, "libkie_trace.so")
-SOURCES = ["monokernel.cu", "kie_host.cu"]
-HEADERS = ["kie_internal.h", os.path.join("..", "..", "include", "kie.h")]
+SOURCES = ["monokernel.cu", "kie_host.cu", "prefill.cu"]
+HEADERS = ["kie_internal.h", "prefill.h", os.path.join("..", "..", "include", "kie.h")]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",

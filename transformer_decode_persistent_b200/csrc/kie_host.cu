@@ -23,6 +23,7 @@
 
 #include "../../include/kie.h"
 #include "kie_internal.h"
+#include "prefill.h"
 
 namespace kie {
 int kernel_smem_bytes(int vec_floats, int n_desc, int n_stages, int stage_bytes);
@@ -76,6 +77,16 @@ struct kie_ctx {
   int64_t launches = 0;
   int64_t stream_bytes = 0;
   std::string err;
+  // tensor-core prompt prefill (dense models): row-major layer matrices in
+  // the packed row orders (q/k/v RoPE pairs and gate/up pairs adjacent),
+  // activation buffers for one chunk, and their tensor maps
+  bool pf_ready = false;
+  __half *pf_w[4] = {nullptr, nullptr, nullptr, nullptr};  // [L][rows][K]: q/k/v, o, gate/up, down
+  float *pf_x = nullptr, *pf_q = nullptr;
+  __half *pf_xh = nullptr, *pf_xl = nullptr, *pf_oh = nullptr, *pf_ol = nullptr, *pf_hh = nullptr, *pf_hl = nullptr;
+  int *pf_tok = nullptr, *pf_err = nullptr;
+  std::vector<CUtensorMap> pf_wmap;  // [L][4]
+  CUtensorMap pf_map_xh{}, pf_map_xl{}, pf_map_oh{}, pf_map_ol{}, pf_map_hh{}, pf_map_hl{};
 };
 
 namespace {
@@ -431,6 +442,104 @@ kie_status validate_config(const kie_config& k) {
 }
 
 }  // namespace
+
+// Buffers and tensor maps of the tensor-core prefill (dense models), once the
+// prefill weights exist.
+static kie_status prefill_setup(kie_ctx* c) {
+  using namespace kie::pf;
+  const kie_config& k = c->cfg;
+  const int d = k.d_model, hq = k.n_heads, hk = k.n_kv_heads, dh = k.head_dim, L = k.n_layers, ff = k.ffn;
+  kie_status s;
+  if (!c->pf_x) {
+    if ((s = dalloc(c, &c->pf_x, (size_t)kChunk * d * 4)) || (s = dalloc(c, &c->pf_q, (size_t)kChunk * hq * dh * 4)) ||
+        (s = dalloc(c, &c->pf_xh, (size_t)kChunk * d * 2)) || (s = dalloc(c, &c->pf_xl, (size_t)kChunk * d * 2)) ||
+        (s = dalloc(c, &c->pf_oh, (size_t)kChunk * hq * dh * 2)) ||
+        (s = dalloc(c, &c->pf_ol, (size_t)kChunk * hq * dh * 2)) ||
+        (s = dalloc(c, &c->pf_hh, (size_t)kChunk * ff * 2)) || (s = dalloc(c, &c->pf_hl, (size_t)kChunk * ff * 2)) ||
+        (s = dalloc(c, &c->pf_tok, (size_t)kChunk * 4)) || (s = dalloc(c, &c->pf_err, 16)))
+      return s;
+    // rows past a chunk's length are read by the last GEMM tile (their
+    // columns are discarded); keep them finite
+    CUDA_TRY(c, cudaMemset(c->pf_xh, 0, (size_t)kChunk * d * 2));
+    CUDA_TRY(c, cudaMemset(c->pf_xl, 0, (size_t)kChunk * d * 2));
+    CUDA_TRY(c, cudaMemset(c->pf_oh, 0, (size_t)kChunk * hq * dh * 2));
+    CUDA_TRY(c, cudaMemset(c->pf_ol, 0, (size_t)kChunk * hq * dh * 2));
+    CUDA_TRY(c, cudaMemset(c->pf_hh, 0, (size_t)kChunk * ff * 2));
+    CUDA_TRY(c, cudaMemset(c->pf_hl, 0, (size_t)kChunk * ff * 2));
+    CUDA_TRY(c, cudaMemset(c->pf_err, 0, 16));
+  }
+  bool ok = make_map(&c->pf_map_xh, c->pf_xh, kChunk, d, kBN) && make_map(&c->pf_map_xl, c->pf_xl, kChunk, d, kBN) &&
+            make_map(&c->pf_map_oh, c->pf_oh, kChunk, hq * dh, kBN) &&
+            make_map(&c->pf_map_ol, c->pf_ol, kChunk, hq * dh, kBN) &&
+            make_map(&c->pf_map_hh, c->pf_hh, kChunk, ff, kBN) && make_map(&c->pf_map_hl, c->pf_hl, kChunk, ff, kBN);
+  const int prow[4] = {(hq + 2 * hk) * dh, d, 2 * ff, d};
+  const int pk[4] = {d, hq * dh, d, ff};
+  c->pf_wmap.assign((size_t)L * 4, CUtensorMap{});
+  for (int l = 0; l < L && ok; ++l)
+    for (int m = 0; m < 4 && ok; ++m)
+      ok = make_map(&c->pf_wmap[(size_t)l * 4 + m], c->pf_w[m] + (size_t)l * prow[m] * pk[m], prow[m], pk[m], kBM);
+  if (!ok) return fail(c, KIE_ERR_CUDA, "tensor map encoding for the prefill failed");
+  c->pf_ready = true;
+  return KIE_OK;
+}
+
+// Forward the committed prompt tokens `seq` at positions pos .. pos + n - 1
+// through the tensor-core path, filling the KV cache (one chunk of up to
+// kChunk tokens at a time; each chunk attends to the cache of the earlier ones).
+static kie_status prefill_tc(kie_ctx* c, const std::vector<int32_t>& seq, cudaStream_t st) {
+  using namespace kie::pf;
+  const kie_config& k = c->cfg;
+  const int d = k.d_model, hq = k.n_heads, hk = k.n_kv_heads, dh = k.head_dim, L = k.n_layers, ff = k.ffn;
+  const int qkv_rows = (hq + 2 * hk) * dh;
+  CUDA_TRY(c, cudaMemsetAsync(c->pf_err, 0, 4, st));
+  for (size_t c0 = 0; c0 < seq.size(); c0 += kChunk) {
+    const int T = (int)std::min<size_t>(kChunk, seq.size() - c0);
+    const int p0 = c->pos + (int)c0;
+    CUDA_TRY(c, cudaMemcpyAsync(c->pf_tok, seq.data() + c0, (size_t)T * 4, cudaMemcpyHostToDevice, st));
+    CUDA_TRY(c, embed(c->pf_tok, c->embed, c->pf_x, T, d, st));
+    for (int l = 0; l < L; ++l) {
+      const CUtensorMap* W = &c->pf_wmap[(size_t)l * 4];
+      CUDA_TRY(c, rmsnorm_split(c->pf_x, c->attn_norm + (size_t)l * d, c->pf_xh, c->pf_xl, T, d, k.rms_eps, st));
+      GemmArgs g{};
+      g.err = c->pf_err;
+      g.M = qkv_rows; g.N = T; g.K = d; g.epi = EPI_QKV;
+      g.q = c->pf_q; g.kcache = c->kcache; g.vcache = c->vcache; g.rope = c->rope;
+      g.layer = l; g.hq = hq; g.hk = hk; g.dh = dh; g.max_ctx = k.max_ctx; g.pos0 = p0;
+      CUDA_TRY(c, gemm(W[0], c->pf_map_xh, c->pf_map_xl, g, st));
+      c->launches += 2;
+      if (l == L - 1) break;  // later positions need only this layer's K and V
+      AttnArgs at{c->pf_q, c->kcache, c->vcache, c->pf_oh, c->pf_ol, T, p0, l, hq, hk, dh, k.max_ctx};
+      CUDA_TRY(c, attention(at, st));
+      GemmArgs o{};
+      o.err = c->pf_err;
+      o.M = d; o.N = T; o.K = hq * dh; o.epi = EPI_RESID; o.x = c->pf_x;
+      CUDA_TRY(c, gemm(W[1], c->pf_map_oh, c->pf_map_ol, o, st));
+      CUDA_TRY(c, rmsnorm_split(c->pf_x, c->mlp_norm + (size_t)l * d, c->pf_xh, c->pf_xl, T, d, k.rms_eps, st));
+      GemmArgs u{};
+      u.err = c->pf_err;
+      u.M = 2 * ff; u.N = T; u.K = d; u.epi = EPI_SWIGLU; u.h_hi = c->pf_hh; u.h_lo = c->pf_hl; u.ff = ff;
+      CUDA_TRY(c, gemm(W[2], c->pf_map_xh, c->pf_map_xl, u, st));
+      GemmArgs w{};
+      w.err = c->pf_err;
+      w.M = d; w.N = T; w.K = ff; w.epi = EPI_RESID; w.x = c->pf_x;
+      CUDA_TRY(c, gemm(W[3], c->pf_map_hh, c->pf_map_hl, w, st));
+      c->launches += 5;
+    }
+    c->launches += 1;
+  }
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) {
+    c->poisoned = true;
+    return fail(c, KIE_ERR_CUDA, "prefill kernels failed: %s", cudaGetErrorString(e));
+  }
+  int err = 0;
+  CUDA_TRY(c, cudaMemcpy(&err, c->pf_err, 4, cudaMemcpyDeviceToHost));
+  if (err) {
+    c->poisoned = true;
+    return fail(c, KIE_ERR_TIMEOUT, "prefill GEMM wait gave up; context poisoned");
+  }
+  return KIE_OK;
+}
 
 extern "C" {
 
@@ -830,6 +939,28 @@ kie_status kie_load_weights(kie_ctx* c, const kie_tensor* tensors, int n, void* 
     dfree(c, staging);
     return ps;
   }
+  // the prefill's row-major copies of the layer matrices (dense models)
+  for (int i = 0; i < 4; ++i) { dfree(c, c->pf_w[i]); c->pf_w[i] = nullptr; }
+  c->pf_ready = false;
+  if (!moe) {
+    const int prow[4] = {(hq + 2 * hk) * dh, d, 2 * k.ffn, d};
+    const int pk[4] = {d, hq * dh, d, k.ffn};
+    for (int m = 0; m < 4 && ps == KIE_OK; ++m) {
+      if ((ps = dalloc(c, &c->pf_w[m], (size_t)L * prow[m] * pk[m] * 2))) break;
+      for (int l = 0; l < L && ps == KIE_OK; ++l) {
+        for (int r = 0; r < prow[m]; ++r) {
+          hsrc.push_back((unsigned long long)rowptr(l, m, r));
+          hdst.push_back((unsigned long long)(c->pf_w[m] + ((size_t)l * prow[m] + r) * pk[m]));
+          hn.push_back(pk[m] / 8);
+        }
+        ps = flush();
+      }
+    }
+    if (ps != KIE_OK) {
+      dfree(c, staging);
+      return ps;
+    }
+  }
   dfree(c, dsrc); dfree(c, ddst); dfree(c, dn);
 
   // descriptors and the small tensors kept outside the tape
@@ -869,6 +1000,10 @@ kie_status kie_load_weights(kie_ctx* c, const kie_tensor* tensors, int n, void* 
   }
   sb += (int64_t)k.vocab * d * 2 + (2LL * L + 1) * d * 2 + (int64_t)d * 2;
   c->stream_bytes = sb;
+  if (!moe) {
+    kie_status s2 = prefill_setup(c);
+    if (s2 != KIE_OK) return s2;
+  }
   c->loaded = true;
   c->pos = 0;
   c->pending = -1;
@@ -987,10 +1122,22 @@ kie_status kie_prefill(kie_ctx* c, const int32_t* tokens, int n, void* stream) {
                 c->cfg.max_ctx);
   cudaSetDevice(c->device);
   cudaStream_t st = (cudaStream_t)stream;
-  const int kChunk = 8192;  // bounds the barrier counter and the flag epochs of one launch
   const int32_t new_pending = tokens[n - 1];
-  size_t i0 = 0;
   const int32_t pos_before = c->pos, pend_before = c->pending;
+  if (c->pf_ready) {
+    // dense models: the chunked tensor-core prefill
+    kie_status s = prefill_tc(c, seq, st);
+    if (s != KIE_OK) {
+      if (!c->poisoned) { c->pos = pos_before; c->pending = pend_before; }
+      return s;
+    }
+    c->pos += (int32_t)seq.size();
+    c->pending = new_pending;
+    return KIE_OK;
+  }
+  // MoE models: the decode kernel in forced-token mode, one position per step
+  const int kChunk = 8192;  // bounds the barrier counter and the flag epochs of one launch
+  size_t i0 = 0;
   while (i0 < seq.size()) {
     const int m = (int)std::min<size_t>(kChunk, seq.size() - i0);
     // forced[i] = token fed after step i

@@ -47,6 +47,8 @@ constexpr int kErrTimeout = -5;  // KIE_ERR_TIMEOUT
 constexpr int kErrDevice = -6;   // KIE_ERR_DEVICE
 
 constexpr int kRouteRing = 8;  // routing decisions kept for lagging issuer lanes
+constexpr int kRopeStage = 128; // RoPE pairs whose coefficients are staged in shared memory
+constexpr int kAttnOneChunk = 2; // up to this many 224-position blocks, a KV head stays in one CTA
 
 struct SmemCtl {
   uint64_t full[kMaxStages];
@@ -58,6 +60,8 @@ struct SmemCtl {
   int route_e[kRouteRing][kMaxTopK];
   float route_w[kMaxTopK];
   float red[64];
+  float ssq[kConsumerWarps];  // per-warp sums of squares of the last RMSNorm input
+  float2 rcs[kRopeStage];     // RoPE (cos, sin) of this CTA's first q/k pairs at this step's position
   Cand wcand[kConsumerWarps];
   unsigned bcast;
   // this CTA's rows of the residual stream: the output projection and the
@@ -389,8 +393,15 @@ __device__ __forceinline__ AttnPlan attn_plan(int pos, int hk, int grid) {
   constexpr int kUnitMin = kConsumerWarps * kAttnSub;
   AttnPlan a;
   a.T = pos + 1;
-  int per = (int)(((long long)a.T * hk + grid - 1) / grid);
-  per = ((max(per, kUnitMin) + kUnitMin - 1) / kUnitMin) * kUnitMin;
+  int per;
+  if (a.T <= kAttnOneChunk * kUnitMin) {
+    // short context: each KV head in one CTA, so no cross-CTA merge of
+    // chunk partials (a merge costs two dependent L2 round trips)
+    per = ((a.T + kUnitMin - 1) / kUnitMin) * kUnitMin;
+  } else {
+    per = (int)(((long long)a.T * hk + grid - 1) / grid);
+    per = ((max(per, kUnitMin) + kUnitMin - 1) / kUnitMin) * kUnitMin;
+  }
   a.per = per;
   a.pw = per / kConsumerWarps;
   a.nsb = a.pw / kAttnSub;
@@ -648,17 +659,6 @@ struct Consumer {
       : P(p), sc(s), part(pa), vec(v), ring(r), tid(threadIdx.x), warp(threadIdx.x >> 5),
         lane(threadIdx.x & 31), dc(d) {}
 
-  __device__ float block_sum(float v) {
-    v = warp_sum(v);
-    if (lane == 0) sc->red[warp] = v;
-    cbar();
-    float t = 0.f;
-#pragma unroll
-    for (int i = 0; i < kConsumerWarps; ++i) t += sc->red[i];
-    cbar();
-    return t;
-  }
-
   __device__ __forceinline__ int ap_nchk(int pos) const { return attn_plan(pos, P.hk, gridDim.x).nchk; }
 
   // Phase trace (KIE_TRACE builds): per CTA and step, one record of four
@@ -716,55 +716,139 @@ struct Consumer {
     return vec + ((i & 4) ? P.xplane : 0) + ((i >> 3) << 2);
   }
 
+  // The flagged words src[i..i+4) for the kLoadBatch groups i = base + b *
+  // kConsumerThreads * 4 (those below n), once they carry epoch ep, into v.
+  // All of the batch's loads are issued before any epoch is checked, and the
+  // groups still stale are re-polled together, so a thread waits about one L2
+  // round trip per batch instead of one per group. Bounded: on abort or
+  // deadline it flags the CTA and leaves zeros.
+  static constexpr int kLoadBatch = 8;
+  __device__ __forceinline__ void fetch_batch(const unsigned long long* src, unsigned ep, int n, int base,
+                                              float4 (&v)[kLoadBatch]) {
+    unsigned long long w[kLoadBatch][4];
+#pragma unroll
+    for (int b = 0; b < kLoadBatch; ++b) {
+      const int i = base + b * kConsumerThreads * 4;
+      w[b][0] = w[b][1] = w[b][2] = w[b][3] = (unsigned long long)ep << 32;
+      if (i < n) {
+        ld_flag2(src + i, w[b][0], w[b][1]);
+        ld_flag2(src + i + 2, w[b][2], w[b][3]);
+      }
+    }
+    unsigned long long t0 = 0;
+    for (unsigned it = 0;; ++it) {
+      bool stale = false;
+#pragma unroll
+      for (int b = 0; b < kLoadBatch; ++b) {
+        const int i = base + b * kConsumerThreads * 4;
+        if (fepoch(w[b][0]) != ep || fepoch(w[b][1]) != ep || fepoch(w[b][2]) != ep || fepoch(w[b][3]) != ep) {
+          stale = true;
+          ld_flag2(src + i, w[b][0], w[b][1]);
+          ld_flag2(src + i + 2, w[b][2], w[b][3]);
+        }
+      }
+      if (!stale) break;
+      if (it == 0) {
+        t0 = gtimer();
+      } else if ((it & 31) == 0) {
+        bool give_up = false;
+        if (sc->abort || ld_relaxed(&P.ctrl->abort)) {
+          give_up = true;
+        } else if (gtimer() - t0 > P.timeout_ns) {
+          record_error(P, kErrTimeout, 6, step);
+          give_up = true;
+        }
+        if (give_up) {
+          sc->abort = 1;
+#pragma unroll
+          for (int b = 0; b < kLoadBatch; ++b) v[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+          return;
+        }
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < kLoadBatch; ++b) v[b] = make_float4(fval(w[b][0]), fval(w[b][1]), fval(w[b][2]), fval(w[b][3]));
+  }
+
   // vec = the flagged vector src[0..n) of epoch ep (n a multiple of 8), once
   // its producers have written it
   __device__ void load_vec(const unsigned long long* src, unsigned ep, int n) {
-    for (int i = tid * 4; i < n; i += kConsumerThreads * 4) *reinterpret_cast<float4*>(xv(i)) = wait4(src + i, ep);
+    for (int base = tid * 4; base < n; base += kConsumerThreads * 4 * kLoadBatch) {
+      float4 v[kLoadBatch];
+      fetch_batch(src, ep, n, base, v);
+#pragma unroll
+      for (int b = 0; b < kLoadBatch; ++b) {
+        const int i = base + b * kConsumerThreads * 4;
+        if (i < n) *reinterpret_cast<float4*>(xv(i)) = v[b];
+      }
+    }
     cbar();
   }
 
   // Start copying the next RMSNorm gain into the shared gain buffer
-  // (cp.async, no registers held); load_norm waits for it. Issued right after
-  // the previous load_norm, so the copy overlaps a whole phase.
+  // (cp.async, no registers held); load_norm waits for it. Each thread copies
+  // the four gains of exactly the elements it will scale in load_norm, so
+  // waiting for its own copies is enough. Issued right after the previous
+  // load_norm, so the copy overlaps a whole phase.
   __device__ void prefetch_gain(const __half* g) {
     const uint32_t gb = su32(vec + P.gbuf_off);
-    for (int i = tid * 8; i < P.d; i += kConsumerThreads * 8)
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(gb + i * 2), "l"(g + i) : "memory");
+    for (int i = tid * 4; i < P.d; i += kConsumerThreads * 4)
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(gb + i * 2), "l"(g + i) : "memory");
     asm volatile("cp.async.commit_group;" ::: "memory");
   }
 
-  // vec = RMSNorm(src) * gain, src either the flagged residual stream of epoch
-  // ep or an fp16 embedding row; the gain was prefetched into the gain buffer
-  // by prefetch_gain.
+  // vec = gain * x, with x either the flagged residual stream of epoch ep or
+  // an fp16 embedding row (the gain was prefetched by prefetch_gain). RMSNorm's
+  // factor 1/sqrt(mean(x^2) + eps) is a scalar, so it is applied to the GEMV
+  // outputs in the epilogue (norm_scale) instead of to x: the tiles start
+  // right after the load, and this CTA's sum of squares travels through the
+  // one barrier the load needs anyway.
   __device__ void load_norm(const unsigned long long* srcf, unsigned ep, const __half* srch, int n) {
-    float ss = 0.f;
-    for (int i = tid * 4; i < n; i += kConsumerThreads * 4) {
-      float4 v;
-      if (srcf) {
-        v = wait4(srcf + i, ep);
-      } else {
-        const uint2 raw = *reinterpret_cast<const uint2*>(srch + i);
-        const float2 lo = h2f2(raw.x), hi = h2f2(raw.y);
-        v = make_float4(lo.x, lo.y, hi.x, hi.y);
-      }
-      *reinterpret_cast<float4*>(xv(i)) = v;
-      ss = fmaf(v.x, v.x, ss);
-      ss = fmaf(v.y, v.y, ss);
-      ss = fmaf(v.z, v.z, ss);
-      ss = fmaf(v.w, v.w, ss);
-    }
     asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's gain copies
-    const float tot = block_sum(ss);                   // (its barrier publishes all of them)
-    const float inv = 1.0f / sqrtf(tot / (float)n + P.eps);
     const __half* gb = reinterpret_cast<const __half*>(vec + P.gbuf_off);
-    for (int i = tid * 4; i < n; i += kConsumerThreads * 4) {
-      const uint2 g = *reinterpret_cast<const uint2*>(gb + i);
-      const float2 g0 = h2f2(g.x), g1 = h2f2(g.y);
-      float4* xp = reinterpret_cast<float4*>(xv(i));
-      const float4 v = *xp;
-      *xp = make_float4(v.x * inv * g0.x, v.y * inv * g0.y, v.z * inv * g1.x, v.w * inv * g1.y);
+    float ss = 0.f;
+    for (int base = tid * 4; base < n; base += kConsumerThreads * 4 * kLoadBatch) {
+      float4 v[kLoadBatch];
+      if (srcf) {
+        fetch_batch(srcf, ep, n, base, v);
+      } else {
+#pragma unroll
+        for (int b = 0; b < kLoadBatch; ++b) {
+          const int i = base + b * kConsumerThreads * 4;
+          v[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (i < n) {
+            const uint2 raw = *reinterpret_cast<const uint2*>(srch + i);
+            const float2 lo = h2f2(raw.x), hi = h2f2(raw.y);
+            v[b] = make_float4(lo.x, lo.y, hi.x, hi.y);
+          }
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < kLoadBatch; ++b) {
+        const int i = base + b * kConsumerThreads * 4;
+        if (i < n) {
+          const float4 x = v[b];
+          ss = fmaf(x.x, x.x, ss);
+          ss = fmaf(x.y, x.y, ss);
+          ss = fmaf(x.z, x.z, ss);
+          ss = fmaf(x.w, x.w, ss);
+          const uint2 g = *reinterpret_cast<const uint2*>(gb + i);
+          const float2 g0 = h2f2(g.x), g1 = h2f2(g.y);
+          *reinterpret_cast<float4*>(xv(i)) = make_float4(x.x * g0.x, x.y * g0.y, x.z * g1.x, x.w * g1.y);
+        }
+      }
     }
+    ss = warp_sum(ss);
+    if (lane == 0) sc->ssq[warp] = ss;
     cbar();
+  }
+
+  // 1/sqrt(mean(x^2) + eps) of the vector the last load_norm read
+  __device__ __forceinline__ float norm_scale() const {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) t += sc->ssq[w];
+    return 1.0f / sqrtf(t / (float)P.d + P.eps);
   }
 
   // Consume one segment's tiles; partial sums land in part[pbase + row*pstride + kjbase + kj].
@@ -1180,6 +1264,21 @@ struct Consumer {
     else attention<64>(l, pos);
   }
 
+  // Copy the RoPE coefficients of this CTA's first kRopeStage q/k row pairs at
+  // position pos into shared memory (cp.async; load_norm's wait covers it).
+  // The thread that copies pair j is the one whose epilogue rotates it.
+  __device__ void stage_rope(const SegDesc& sd, int pos) {
+    const int dh = P.dh, npairs = min(sd.nrows / 2, kRopeStage);
+    const float2* rp = P.rope + (size_t)pos * (dh / 2);
+    for (int j = tid; j < npairs; j += kConsumerThreads) {
+      const int r = sd.row0 + 2 * j;
+      const int H = r / dh, pi = (r - H * dh) / 2;
+      if (H < P.hq + P.hk)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(su32(&sc->rcs[j])), "l"(rp + pi) : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+
   // q/k/v epilogue. The q/k/v rows are packed so that every CTA owns whole
   // RoPE pairs (dims i and i + dh/2 of one head are adjacent virtual rows), so
   // RoPE is applied here: q is rotated and pre-scaled by 1/sqrt(dh), k is
@@ -1190,13 +1289,14 @@ struct Consumer {
     const int dh = P.dh, half = P.dh / 2, hq = P.hq, hk = P.hk;
     const float2* rp = P.rope + (size_t)pos * half;
     const float scale = 1.0f / sqrtf((float)dh);
+    const float inv = norm_scale();
     const unsigned ep = epoch(l);
     for (int j = tid; j < sd.nrows / 2; j += kConsumerThreads) {
       const int r = sd.row0 + 2 * j;
       const int H = r / dh, pi = (r - H * dh) / 2;
-      const float ya = row_sum(2 * j, stride), yb = row_sum(2 * j + 1, stride);
+      const float ya = row_sum(2 * j, stride) * inv, yb = row_sum(2 * j + 1, stride) * inv;
       if (H < hq + hk) {
-        const float2 cs = rp[pi];
+        const float2 cs = j < kRopeStage ? sc->rcs[j] : rp[pi];
         const float a = ya * cs.x - yb * cs.y, b = ya * cs.y + yb * cs.x;
         if (H < hq) {
           st_flag(P.fq + (size_t)H * dh + pi, a * scale, ep);
@@ -1239,12 +1339,15 @@ struct Consumer {
   // SwiGLU epilogue over interleaved (gate, up) rows: h[hoff + row0/2 + j] = w * silu(g) * u
   __device__ void epi_swiglu(const SegDesc& sd, int pbase, int stride, int hoff, float w, unsigned ep) {
     const int npairs = sd.nrows / 2;
+    const float inv = norm_scale();
     for (int j = tid; j < npairs; j += kConsumerThreads) {
       float yg = 0.f, yu = 0.f;
       for (int k = 0; k < stride; ++k) {
         yg += part[pbase + (2 * j) * stride + k];
         yu += part[pbase + (2 * j + 1) * stride + k];
       }
+      yg *= inv;
+      yu *= inv;
       st_flag(P.fh + hoff + sd.row0 / 2 + j, w * silu(yg) * yu, ep);
     }
   }
@@ -1261,7 +1364,7 @@ struct Consumer {
                  *reinterpret_cast<const float4*>(xv(c * 8 + 4)), a);
       }
       a = warp_sum(a);
-      if (lane == 0) part[e] = a;
+      if (lane == 0) part[e] = a * norm_scale();
     }
     cbar();
     if (tid == 0) {
@@ -1326,6 +1429,7 @@ struct Consumer {
         // ---- 1. input vector
         switch (kind) {
           case PH_QKV:
+            stage_rope(dc.at(l, 0), pos);
             if (l == 0) load_norm(nullptr, 0u, erow, P.d);
             else load_norm(P.fx + P.d, epoch(l - 1), nullptr, P.d);
             prefetch_gain(P.mlp_norm + (size_t)l * P.d);
@@ -1447,10 +1551,11 @@ struct Consumer {
   // LM-head epilogue: logits (optional copy out) and this CTA's greedy candidate.
   __device__ void epi_lm(const SegDesc& dl) {
     const int stride = P.shp[SK_LM].nk;
+    const float inv = norm_scale();
     float v1 = -INFINITY, v2 = -INFINITY;
     int i1 = INT_MAX;
     for (int r = tid; r < dl.nrows; r += kConsumerThreads) {
-      const float y = row_sum(r, stride);
+      const float y = row_sum(r, stride) * inv;
       const int row = dl.row0 + r;
       if (P.logits_out) P.logits_out[(size_t)step * P.V + row] = y;
       cand_merge(v1, i1, v2, y, row, -INFINITY);

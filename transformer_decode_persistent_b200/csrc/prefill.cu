@@ -1,0 +1,437 @@
+// Chunked prompt prefill for dense models on B200 (sm_100a) tensor cores.
+//
+// Before the first decode step the engine must hold the KV cache of every
+// prompt position. The pages' persistent kernel covers the per-token decode
+// step ("メモリの壁を打破する：標準的なGPUで3,000 tokens/sの推論を実現する", section
+// "1. The Monokernel Runtime"); a long prompt is a different workload that the
+// pages leave open ("Kog、より深いGPU最適化でAI推論を高速化できると賭ける", section
+// "Kogのベンチマークでは決着しないこと": long prompts and contexts are the untested
+// case). Processed as chunks of up to kChunk tokens, the prompt's projections
+// are dense contractions, so they run on the 5th-generation tensor cores:
+//
+//  * gemm_kernel: D[128 weight rows x 128 tokens] = W[rows, K] . X[tokens, K]^T
+//    with tcgen05.mma (kind::f16, fp32 accumulator in tensor memory). TMA
+//    loads 64-wide K slices of W and X with 128-byte swizzle into a 4-stage
+//    shared-memory ring; one thread issues the MMAs, another the loads, and
+//    four warps read the accumulator back with tcgen05.ld for a fused
+//    epilogue. The activations enter as two fp16 parts, hi = fp16(x) and
+//    lo = fp16(x - hi), accumulated into the same fp32 accumulator, so the
+//    products carry about 22 bits of the fp32 activation (a single fp16
+//    operand would carry 11); the weights are fp16 already.
+//  * epilogues: q/k/v (RoPE on adjacent row pairs, q scaled by 1/sqrt(dh), K
+//    and V appended to the fp16 cache the decode kernel reads), residual add
+//    (output and down projections) and SwiGLU (gate/up rows interleaved).
+//  * rmsnorm_split_kernel, embed_kernel and attention_kernel (causal softmax
+//    attention over the cache in fp32 on the CUDA cores).
+//
+// The last layer's attention, output projection and FFN are skipped: a
+// prompt position contributes nothing but its K and V.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "prefill.h"
+
+namespace kie {
+namespace pf {
+
+// ---------------------------------------------------------------- GEMM
+
+constexpr int kStageBytes = kTileA + 2 * kTileB;
+constexpr unsigned kSpinLimit = 1u << 28;  // bounded mbarrier waits (several seconds)
+
+__device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ bool mbar_try(uint32_t b, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(b), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait; on giving up it records an error and returns false.
+__device__ __forceinline__ bool mbar_wait(uint32_t b, unsigned parity, int* err) {
+  for (unsigned i = 0; i < kSpinLimit; ++i)
+    if (mbar_try(b, parity)) return true;
+  atomicExch(err, 1);
+  return false;
+}
+
+// K-major operand tile in shared memory as TMA writes it with 128-byte
+// swizzle: rows of 64 fp16 (128 bytes), 8-row groups 1024 bytes apart. The
+// descriptor fields: start address >> 4 (bits 0-13), leading byte offset 1
+// (unused by swizzled K-major layouts), stride byte offset 1024 >> 4 (bits
+// 32-45), descriptor version 1 (bits 46-47), swizzle mode 128B = 2 (bits
+// 61-63). A K step of 16 elements advances the start address by 32 bytes.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor of kind::f16: fp32 accumulator (bits 4-5 = 1), A and
+// B fp16 (formats 0), both K-major, N >> 3 at bits 17-22, M >> 4 at bits 24-28.
+constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+
+__device__ __forceinline__ void tma2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(map), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma(uint32_t tmem, uint64_t a, uint64_t b, bool acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+      "l"(a), "l"(b), "r"(kIdesc), "r"((unsigned)acc)
+      : "memory");
+}
+__device__ __forceinline__ void commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
+
+__device__ __forceinline__ void split_store(__half* hi, __half* lo, size_t i, float v) {
+  const __half h = __float2half_rn(v);
+  hi[i] = h;
+  lo[i] = __float2half_rn(v - __half2float(h));
+}
+
+// Epilogue for one 32-token slice of the accumulator: this thread holds
+// D[row][n .. n+32) (row = this thread's weight row). Rows beyond M and
+// tokens beyond N are skipped; the lane-pair exchanges run on every lane.
+__device__ __forceinline__ void epilogue(const GemmArgs& a, int row, int n, const float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+  const bool row_ok = row < a.M;
+  if (a.epi == EPI_RESID) {
+    if (!row_ok) return;
+#pragma unroll 4
+    for (int j = 0; j < 32; ++j)
+      if (n + j < a.N) a.x[(size_t)(n + j) * a.M + row] += v[j];
+    return;
+  }
+  if (a.epi == EPI_SWIGLU) {
+    // rows 2j (gate) and 2j+1 (up) sit on lanes 2i and 2i+1 of one warp
+#pragma unroll 4
+    for (int j = 0; j < 32; ++j) {
+      const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
+      if (row_ok && !(lane & 1) && n + j < a.N) {
+        const float h = silu(v[j]) * other;
+        split_store(a.h_hi, a.h_lo, (size_t)(n + j) * a.ff + row / 2, h);
+      }
+    }
+    return;
+  }
+  // EPI_QKV: virtual rows of a head run dims 0, dh/2, 1, dh/2 + 1, ... so a
+  // RoPE pair (i, i + dh/2) sits on lanes 2p and 2p+1
+  const int dh = a.dh, H = row / dh, vr = row - H * dh, pi = vr >> 1;
+  const int dim = (vr & 1) ? pi + dh / 2 : pi;
+  const float scale = rsqrtf((float)dh);
+#pragma unroll 2
+  for (int j = 0; j < 32; ++j) {
+    const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
+    const int t = n + j;
+    if (!row_ok || t >= a.N) continue;
+    const int pos = a.pos0 + t;
+    if (H < a.hq + a.hk) {
+      const float2 cs = a.rope[(size_t)pos * (dh / 2) + pi];
+      const float x0 = (vr & 1) ? other : v[j], x1 = (vr & 1) ? v[j] : other;
+      const float r = (vr & 1) ? (x0 * cs.y + x1 * cs.x) : (x0 * cs.x - x1 * cs.y);
+      if (H < a.hq) {
+        a.q[(size_t)t * a.hq * dh + (size_t)H * dh + dim] = r * scale;
+      } else {
+        a.kcache[((size_t)(a.layer * a.hk + (H - a.hq)) * a.max_ctx + pos) * dh + dim] = __float2half_rn(r);
+      }
+    } else {
+      a.vcache[((size_t)(a.layer * a.hk + (H - a.hq - a.hk)) * a.max_ctx + pos) * dh + dim] = __float2half_rn(v[j]);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmBh,
+                const __grid_constant__ CUtensorMap tmBl, const GemmArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* accf = empty + kStages;
+  uint32_t* taddr_s = reinterpret_cast<uint32_t*>(accf + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kBM, n0 = blockIdx.y * kBN;
+  const int nkb = (a.K + kBK - 1) / kBK;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(&full[s])));
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(&empty[s])));
+    }
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(accf)));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(taddr_s)),
+                 "r"(kBN));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *taddr_s;
+  bool ok = true;
+
+  if (warp == 0 && lane == 0) {
+    // TMA producer
+    int issued = 0;
+    for (int kb = 0; kb < nkb && ok; ++kb) {
+      const int s = kb % kStages;
+      const unsigned r = (unsigned)(kb / kStages);
+      if (r > 0) ok = mbar_wait(su32(&empty[s]), (r - 1) & 1u, a.err);
+      if (!ok) break;
+      ++issued;
+      unsigned char* st = smem + s * kStageBytes;
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(&full[s])), "r"(kStageBytes)
+                   : "memory");
+      tma2d(su32(st), &tmA, kb * kBK, m0, su32(&full[s]));
+      tma2d(su32(st + kTileA), &tmBh, kb * kBK, n0, su32(&full[s]));
+      tma2d(su32(st + kTileA + kTileB), &tmBl, kb * kBK, n0, su32(&full[s]));
+    }
+    // let every copy this thread issued land before the CTA can exit (on the
+    // normal path the MMA issuer has already waited for all of them)
+    for (int kb = issued - 1; kb >= 0 && kb >= issued - kStages; --kb)
+      mbar_wait(su32(&full[kb % kStages]), (unsigned)(kb / kStages) & 1u, a.err);
+  } else if (warp == 1 && lane == 0) {
+    // MMA issuer
+    for (int kb = 0; kb < nkb && ok; ++kb) {
+      const int s = kb % kStages;
+      ok = mbar_wait(su32(&full[s]), (unsigned)(kb / kStages) & 1u, a.err);
+      if (!ok) break;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t sa = su32(smem + s * kStageBytes);
+      const uint64_t da = sdesc(sa), dhi = sdesc(sa + kTileA), dlo = sdesc(sa + kTileA + kTileB);
+#pragma unroll
+      for (int ks = 0; ks < kBK / 16; ++ks) {
+        mma(tmem, da + 2 * ks, dhi + 2 * ks, kb > 0 || ks > 0);
+        mma(tmem, da + 2 * ks, dlo + 2 * ks, true);
+      }
+      commit(su32(&empty[s]));  // the stage is free once these MMAs have read it
+    }
+    commit(su32(accf));  // arrives once every MMA issued above has completed
+  }
+  __syncwarp();
+
+  // epilogue: warp w reads accumulator lanes (rows) 32w .. 32w + 31
+  ok = mbar_wait(su32(accf), 0u, a.err);
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  if (ok) {
+    const int row = m0 + warp * 32 + lane;
+    for (int c = 0; c < kBN; c += 32) {
+      float v[32];
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
+      if (n0 + c < a.N) epilogue(a, row, n0 + c, v);
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kBN));
+}
+
+// ---------------------------------------------------------------- small kernels
+
+// x[t] = E[tok[t]] (fp16 -> fp32), one block per token
+__global__ void embed_kernel(const int* tok, const __half* E, float* x, int d) {
+  const int t = blockIdx.x;
+  const __half* e = E + (size_t)tok[t] * d;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) x[(size_t)t * d + i] = __half2float(e[i]);
+}
+
+// xn = x / sqrt(mean(x^2) + eps) * g, written as fp16 hi and lo parts; one
+// block of 256 threads per token
+__global__ void rmsnorm_split_kernel(const float* x, const __half* g, __half* hi, __half* lo, int d, float eps) {
+  __shared__ float red[8];
+  const int t = blockIdx.x;
+  const float* xr = x + (size_t)t * d;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) ss = fmaf(xr[i], xr[i], ss);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += red[w];
+  const float inv = 1.0f / sqrtf(tot / (float)d + eps);
+  for (int i = threadIdx.x; i < d; i += blockDim.x) split_store(hi, lo, (size_t)t * d + i, xr[i] * inv * __half2float(g[i]));
+}
+
+// Causal attention of T prompt tokens (positions pos0 .. pos0 + T - 1) over
+// the cache of one layer, in fp32: block (query head h, block of kQB tokens);
+// keys stream through shared memory in blocks of kKB with an online softmax.
+// q is rotated and pre-scaled by 1/sqrt(dh). Output as fp16 hi/lo parts
+// [T][hq * dh] (the next GEMM's operand). 256 threads: 8 threads per query
+// token (kQB = 32), each owning dh / 8 output dims.
+constexpr int kQB = 32, kKB = 32;
+template <int DH>
+__global__ void __launch_bounds__(256) attention_kernel(AttnArgs a) {
+  constexpr int DPT = DH / 8;  // output dims per thread
+  __shared__ float qs[kQB][DH + 1];
+  __shared__ __half ks[kKB][DH + 2];
+  __shared__ __half vs[kKB][DH];
+  __shared__ float ps[kQB][kKB + 1];
+  const int h = blockIdx.x, qb = blockIdx.y;
+  const int g = (h * a.hk) / a.hq;
+  const int qi = threadIdx.x >> 3, sub = threadIdx.x & 7;
+  const int t0 = qb * kQB, t = t0 + qi;
+  const bool live = t < a.T;
+  for (int i = threadIdx.x; i < kQB * DH; i += 256) {
+    const int r = i / DH, c = i - r * DH;
+    qs[r][c] = (t0 + r < a.T) ? a.q[(size_t)(t0 + r) * a.hq * DH + (size_t)h * DH + c] : 0.f;
+  }
+  float m = -INFINITY, l = 0.f, acc[DPT];
+#pragma unroll
+  for (int e = 0; e < DPT; ++e) acc[e] = 0.f;
+  const int last = a.pos0 + min(a.T, t0 + kQB) - 1;  // last key any query of this block sees
+  const __half* K = a.kcache + (size_t)(a.layer * a.hk + g) * a.max_ctx * DH;
+  const __half* V = a.vcache + (size_t)(a.layer * a.hk + g) * a.max_ctx * DH;
+  for (int j0 = 0; j0 <= last; j0 += kKB) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < kKB * DH / 2; i += 256) {
+      const int r = (2 * i) / DH, c = 2 * i - r * DH;
+      __half2 kv = __floats2half2_rn(0.f, 0.f), vv = kv;
+      if (j0 + r <= last) {
+        kv = *reinterpret_cast<const __half2*>(K + (size_t)(j0 + r) * DH + c);
+        vv = *reinterpret_cast<const __half2*>(V + (size_t)(j0 + r) * DH + c);
+      }
+      *reinterpret_cast<__half2*>(&ks[r][c]) = kv;
+      *reinterpret_cast<__half2*>(&vs[r][c]) = vv;
+    }
+    __syncthreads();
+    // scores: thread (qi, sub) computes keys sub, sub + 8, ... of the block
+    const int pos = a.pos0 + t;
+    float smax = -INFINITY;
+    for (int jj = sub; jj < kKB; jj += 8) {
+      float s = 0.f;
+#pragma unroll 8
+      for (int c = 0; c < DH; ++c) s = fmaf(qs[qi][c], __half2float(ks[jj][c]), s);
+      s = (live && j0 + jj <= pos) ? s : -INFINITY;
+      ps[qi][jj] = s;
+      smax = fmaxf(smax, s);
+    }
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+    const float mn = fmaxf(m, smax);
+    const float corr = (mn == -INFINITY) ? 1.f : expf(m - mn);
+    float psum = 0.f;
+    for (int jj = sub; jj < kKB; jj += 8) {
+      const float s = ps[qi][jj];
+      const float p = (s == -INFINITY) ? 0.f : expf(s - mn);
+      ps[qi][jj] = p;
+      psum += p;
+    }
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
+    __syncwarp();
+    l = l * corr + psum;
+    m = mn;
+#pragma unroll
+    for (int e = 0; e < DPT; ++e) acc[e] *= corr;
+    for (int jj = 0; jj < kKB; ++jj) {
+      const float p = ps[qi][jj];
+#pragma unroll
+      for (int e = 0; e < DPT; ++e) acc[e] = fmaf(p, __half2float(vs[jj][sub * DPT + e]), acc[e]);
+    }
+  }
+  if (live) {
+    const float inv = 1.0f / l;
+    const size_t base = (size_t)t * a.hq * DH + (size_t)h * DH + sub * DPT;
+#pragma unroll
+    for (int e = 0; e < DPT; ++e) split_store(a.o_hi, a.o_lo, base + e, acc[e] * inv);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    else
+      cudaGetLastError();
+  }
+  return fn;
+}
+
+}  // namespace
+
+bool make_map(CUtensorMap* map, const __half* base, int rows, int cols, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t gemm(const CUtensorMap& A, const CUtensorMap& Bh, const CUtensorMap& Bl, const GemmArgs& a,
+                 cudaStream_t st) {
+  // the shared-memory opt-in is per device; setting it again is harmless
+  static bool attr[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr[dev] = true;
+  }
+  const dim3 grid((a.M + kBM - 1) / kBM, (a.N + kBN - 1) / kBN);
+  gemm_kernel<<<grid, kGemmThreads, kGemmSmem, st>>>(A, Bh, Bl, a);
+  return cudaGetLastError();
+}
+
+cudaError_t embed(const int* tok, const __half* E, float* x, int T, int d, cudaStream_t st) {
+  embed_kernel<<<T, 256, 0, st>>>(tok, E, x, d);
+  return cudaGetLastError();
+}
+
+cudaError_t rmsnorm_split(const float* x, const __half* g, __half* hi, __half* lo, int T, int d, float eps,
+                          cudaStream_t st) {
+  rmsnorm_split_kernel<<<T, 256, 0, st>>>(x, g, hi, lo, d, eps);
+  return cudaGetLastError();
+}
+
+cudaError_t attention(const AttnArgs& a, cudaStream_t st) {
+  const dim3 grid(a.hq, (a.T + kQB - 1) / kQB);
+  if (a.dh == 128) attention_kernel<128><<<grid, 256, 0, st>>>(a);
+  else attention_kernel<64><<<grid, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace pf
+}  // namespace kie
