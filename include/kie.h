@@ -108,6 +108,22 @@ typedef struct {
                                    [grid][trace_cap][2] globaltimer stamps of each
                                    grid barrier's arrival and release; NULL = off */
   int32_t trace_cap;            /* barriers recorded per CTA                          */
+  /* Token choice. temperature = 0 (the default): greedy argmax, lowest index
+     on exact ties. temperature > 0: sampling inside the kernel -- z = logit /
+     temperature; keep the top_k largest z (1 <= top_k <= 64; ties: lower
+     index first); weights exp(z - max z); keep the shortest prefix, in that
+     order, whose cumulative weight reaches top_p (0 < top_p <= 1) of the
+     total; pick the first token whose cumulative weight exceeds u times the
+     kept total. u = (w >> 8) * 2^-24, w the first output word of Philox4x32-10
+     with counter (position of the step's forward, 0, 0, 0) and key (seed low
+     32 bits, seed high 32 bits), so a split decode draws the same numbers.
+     out_tokens gets the chosen token; margins_out still gets the top-1 minus
+     top-2 logit. Errors: INVALID_ARG for a negative temperature, or, when
+     sampling, top_k outside [1, 64] or top_p outside (0, 1]. */
+  float temperature;
+  int32_t top_k;
+  float top_p;
+  uint64_t seed;
 } kie_decode_opts;
 
 /* Static facts about a loaded context, for measurement. */

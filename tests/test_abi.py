@@ -43,10 +43,11 @@ def test_library_exports_every_declared_symbol(L):
 
 def test_struct_layouts_match_header():
     # sizes from the C declarations (LP64): config 12*4 + 2*4; tensor 8+8+16+4(+4 pad);
-    # opts 8*3 + 4*3 (+4 pad) + 8 + 4 (+4 pad); info 6*4 + 4*8
+    # opts 8*3 + 4*3 (+4 pad) + 8 + 4 + 4 (temperature) + 4 (top_k) + 4 (top_p) (+4 pad)
+    # + 8 (seed); info 6*4 + 4*8
     assert ctypes.sizeof(K.kie_config) == 56
     assert ctypes.sizeof(K.kie_tensor) == 40
-    assert ctypes.sizeof(K.kie_decode_opts) == 56
+    assert ctypes.sizeof(K.kie_decode_opts) == 72
     assert ctypes.sizeof(K.kie_info) == 56
     # plan: shape 4*4; range 8 + 2*4; info 2*4 + 8 + 9*16
     assert ctypes.sizeof(K.kie_seg_shape) == 16

@@ -63,8 +63,9 @@ struct kie_ctx {
          *router = nullptr;
   __half *kcache = nullptr, *vcache = nullptr;
   float2* rope = nullptr;
-  float* apart = nullptr;
-  // Ctrl | acnt[L][hk] | flagged scratch (fx, fq, fo, fh, fcand), cleared before every launch
+  unsigned long long* fsamp = nullptr;  // sampling candidates (allocated on first use)
+  size_t fsamp_bytes = 0;
+  // Ctrl | flagged scratch (fx, fq, fo, fh, fcand, attention chunk records), cleared before every launch
   unsigned char* syncblk = nullptr;
   size_t syncblk_bytes = 0;
   int *tok_dev = nullptr, *forced_dev = nullptr;
@@ -380,26 +381,26 @@ kie_status make_plan(kie_ctx* c, const kie_config& k, int G, int sb, Plan& plan)
 // The region cleared before every launch: control block, attention arrival
 // counters and the flagged scratch words (see Params).
 struct SyncLayout {
-  size_t acnt, fx, fq, fo, fh, fcand, total;
+  size_t fx, fq, fo, fh, fcand, apart, total;
 };
 
-SyncLayout sync_layout(const kie_config& k, int grid, int hbuf) {
+SyncLayout sync_layout(const kie_config& k, int grid, int hbuf, int max_chunks) {
   auto a16 = [](size_t b) { return (b + 15) & ~(size_t)15; };
   SyncLayout L{};
   size_t off = a16(sizeof(Ctrl));
-  L.acnt = off;  off = a16(off + (size_t)k.n_layers * k.n_kv_heads * sizeof(unsigned));
   L.fx = off;    off += (size_t)2 * k.d_model * 8;
   L.fq = off;    off += (size_t)(k.n_heads + 2 * k.n_kv_heads) * k.head_dim * 8;
   L.fo = off;    off += (size_t)k.n_heads * k.head_dim * 8;
   L.fh = off;    off += (size_t)hbuf * 8;
   L.fcand = off; off += (size_t)grid * 4 * 8;
+  L.apart = off; off += (size_t)k.n_heads * max_chunks * (k.head_dim + 4) * 8;
   L.total = off;
   return L;
 }
 
 void set_sync_params(Params& P, unsigned char* base, const SyncLayout& L) {
   P.ctrl = reinterpret_cast<Ctrl*>(base);
-  P.acnt = reinterpret_cast<unsigned*>(base + L.acnt);
+  P.apart = reinterpret_cast<unsigned long long*>(base + L.apart);
   P.fx = reinterpret_cast<unsigned long long*>(base + L.fx);
   P.fq = reinterpret_cast<unsigned long long*>(base + L.fq);
   P.fo = reinterpret_cast<unsigned long long*>(base + L.fo);
@@ -630,12 +631,11 @@ kie_status kie_create(const kie_config* cfg, int device, kie_ctx** out) {
         cudaSuccess)
       return bail(fail(c, KIE_ERR_CUDA, "rope table upload failed"));
   }
-  if ((s = dalloc(c, &c->apart, (size_t)hq * c->max_chunks * (dh + 4) * 4)) ||
-      (s = dalloc(c, &c->tok_dev, (size_t)k.max_ctx * 4)) ||
+  if ((s = dalloc(c, &c->tok_dev, (size_t)k.max_ctx * 4)) ||
       (s = dalloc(c, &c->forced_dev, (size_t)k.max_ctx * 4)) ||
       (s = dalloc(c, &c->margins_dev, (size_t)k.max_ctx * 4)))
     return bail(s);
-  c->syncblk_bytes = sync_layout(k, c->grid, c->hbuf).total;
+  c->syncblk_bytes = sync_layout(k, c->grid, c->hbuf, c->max_chunks).total;
   if ((s = dalloc(c, &c->syncblk, c->syncblk_bytes))) return bail(s);
   if (cudaMemset(c->syncblk, 0, c->syncblk_bytes) != cudaSuccess)
     return bail(fail(c, KIE_ERR_CUDA, "memset failed"));
@@ -1025,13 +1025,16 @@ struct Run {
   int fault_cta, fault_barrier;
   uint64_t* trace;
   int trace_cap;
+  float temperature = 0.f, top_p = 1.f;
+  int top_k = 0;
+  uint64_t seed = 0;
 };
 
 // The kernel's parameter block for run `r`, with the per-launch scratch (the
-// region cleared before every launch: control block, arrival counters and
-// flagged words) at `sync_base` and the attention partials at `apart`. Both
-// entry points that launch the kernel build their parameters here.
-Params make_params(const kie_ctx* c, const Run& r, unsigned char* sync_base, float* apart) {
+// region cleared before every launch: control block and flagged words) at
+// `sync_base`. Both entry points that launch the kernel build their
+// parameters here.
+Params make_params(const kie_ctx* c, const Run& r, unsigned char* sync_base) {
   const kie_config& k = c->cfg;
   Params P{};
   P.L = k.n_layers; P.d = k.d_model; P.hq = k.n_heads; P.hk = k.n_kv_heads; P.dh = k.head_dim;
@@ -1044,8 +1047,7 @@ Params make_params(const kie_ctx* c, const Run& r, unsigned char* sync_base, flo
   P.embed = c->embed; P.attn_norm = c->attn_norm; P.mlp_norm = c->mlp_norm;
   P.final_norm = c->final_norm; P.router = c->router;
   P.kcache = c->kcache; P.vcache = c->vcache; P.rope = c->rope;
-  P.apart = apart;
-  set_sync_params(P, sync_base, sync_layout(k, c->grid, c->hbuf));
+  set_sync_params(P, sync_base, sync_layout(k, c->grid, c->hbuf, c->max_chunks));
   P.max_chunks = c->max_chunks;
   P.pos0 = c->pos; P.n_steps = r.n_steps; P.first_token = r.first_token; P.lm_from_step = r.lm_from_step;
   P.forced = r.forced; P.out_tokens = r.out; P.logits_out = r.logits; P.margins_out = r.margins;
@@ -1055,6 +1057,8 @@ Params make_params(const kie_ctx* c, const Run& r, unsigned char* sync_base, flo
   P.n_stages = c->n_stages; P.stage_bytes = c->stage_bytes; P.vec_floats = c->vec_floats;
   P.xplane = c->xplane;
   P.gbuf_off = c->gbuf_off;
+  P.samp_temp = r.temperature; P.samp_p = r.top_p; P.samp_k = r.top_k; P.samp_seed = r.seed;
+  P.fsamp = c->fsamp;
   return P;
 }
 
@@ -1062,10 +1066,10 @@ Params make_params(const kie_ctx* c, const Run& r, unsigned char* sync_base, flo
 // kernel for run `r`, wait for it and read its error record. On success the
 // pending token becomes the kernel's last one (position bookkeeping is the
 // caller's).
-kie_status launch_on(kie_ctx* c, const Run& r, unsigned char* sync_base, size_t sync_bytes, float* apart,
-                     cudaStream_t st) {
-  Params P = make_params(c, r, sync_base, apart);
+kie_status launch_on(kie_ctx* c, const Run& r, unsigned char* sync_base, size_t sync_bytes, cudaStream_t st) {
+  Params P = make_params(c, r, sync_base);
   CUDA_TRY(c, cudaMemsetAsync(sync_base, 0, sync_bytes, st));
+  if (r.temperature > 0.f) CUDA_TRY(c, cudaMemsetAsync(c->fsamp, 0, c->fsamp_bytes, st));
   void* args[] = {&P};
   cudaError_t e = cudaLaunchCooperativeKernel(kernel_entry(), dim3(c->grid), dim3(kThreads), args,
                                               (size_t)c->smem, st);
@@ -1096,7 +1100,7 @@ kie_status launch_on(kie_ctx* c, const Run& r, unsigned char* sync_base, size_t 
 
 // A launch with the context's own scratch.
 kie_status launch(kie_ctx* c, const Run& r, cudaStream_t st) {
-  return launch_on(c, r, c->syncblk, c->syncblk_bytes, c->apart, st);
+  return launch_on(c, r, c->syncblk, c->syncblk_bytes, st);
 }
 
 }  // namespace
@@ -1173,6 +1177,19 @@ kie_status kie_decode(kie_ctx* c, int n, int32_t* out_tokens, const kie_decode_o
   o.fault_barrier = -1;
   if (opts) o = *opts;
   if (o.trace_out && o.trace_cap <= 0) return fail(c, KIE_ERR_INVALID_ARG, "trace_cap must be > 0");
+  if (!(o.temperature >= 0.f) || o.temperature > 1e6f)
+    return fail(c, KIE_ERR_INVALID_ARG, "temperature must be >= 0");
+  if (o.temperature > 0.f) {
+    if (o.top_k < 1 || o.top_k > kSampleK)
+      return fail(c, KIE_ERR_INVALID_ARG, "sampling needs 1 <= top_k <= %d (got %d)", kSampleK, o.top_k);
+    if (!(o.top_p > 0.f && o.top_p <= 1.f)) return fail(c, KIE_ERR_INVALID_ARG, "top_p must be in (0, 1]");
+    if (c->grid > kSampleMaxGrid) return fail(c, KIE_ERR_INVALID_ARG, "sampling supports at most %d CTAs", kSampleMaxGrid);
+    if (!c->fsamp) {
+      c->fsamp_bytes = ((size_t)c->grid * 2 * kSampleK + 4) * 8;
+      kie_status s0 = dalloc(c, &c->fsamp, c->fsamp_bytes);
+      if (s0) return s0;
+    }
+  }
   if (o.trace_out && ptr_device(o.trace_out) != c->device)
     return fail(c, KIE_ERR_INVALID_ARG, "trace_out must be memory of device %d", c->device);
   {
@@ -1216,7 +1233,7 @@ kie_status kie_decode(kie_ctx* c, int n, int32_t* out_tokens, const kie_decode_o
   float* margins = nullptr;
   if (o.margins_out) margins = is_device_ptr(o.margins_out) ? o.margins_out : c->margins_dev;
   Run r{c->pending, n, 0, forced, out_dev ? out_tokens : c->tok_dev, logits, margins, o.timeout_ms,
-        o.fault_cta, o.fault_barrier, o.trace_out, o.trace_cap};
+        o.fault_cta, o.fault_barrier, o.trace_out, o.trace_cap, o.temperature, o.top_p, o.top_k, o.seed};
   kie_status s = launch(c, r, st);
   if (s == KIE_OK) {
     if (!out_dev) {
@@ -1268,7 +1285,7 @@ unsigned char* g_static_ptr[kMaxDevices] = {};
 size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
 
 struct StaticLayout {
-  size_t sync, sync_bytes, apart, total;
+  size_t sync, sync_bytes, total;
 };
 
 StaticLayout static_layout(const kie_ctx* c) {
@@ -1276,9 +1293,8 @@ StaticLayout static_layout(const kie_ctx* c) {
   StaticLayout L{};
   size_t off = 0;
   L.sync = off;
-  L.sync_bytes = sync_layout(k, c->grid, c->hbuf).total;
+  L.sync_bytes = sync_layout(k, c->grid, c->hbuf, c->max_chunks).total;
   off += align256(L.sync_bytes);
-  L.apart = off; off += align256((size_t)k.n_heads * c->max_chunks * (k.head_dim + 4) * 4);
   L.total = off;
   return L;
 }
@@ -1323,7 +1339,7 @@ extern "C" kie_status kie_decode_static(kie_ctx* c, int n, int32_t* out_tokens, 
   // abort flag, the attention arrival counters and the flagged words' epochs
   // must start at zero, which launch_on's clear of the sync region ensures
   const Run r{c->pending, n, 0, nullptr, out_tokens, nullptr, nullptr, 0, -1, -1, nullptr, 0};
-  kie_status s = launch_on(c, r, base + lay.sync, lay.sync_bytes, reinterpret_cast<float*>(base + lay.apart), st);
+  kie_status s = launch_on(c, r, base + lay.sync, lay.sync_bytes, st);
   if (s != KIE_OK) return s;
   c->pos += n;
   return KIE_OK;

@@ -24,6 +24,8 @@ constexpr int kMaxTopK = 4;                            // routed experts per tok
 constexpr int kAttnSub = 32;                           // positions per attention sub-block
 constexpr int kMaxExperts = 64;
 constexpr int kMaxOwnRows = 64;                        // residual rows a CTA keeps in shared memory
+constexpr int kSampleK = 64;                           // largest top-k of in-kernel sampling
+constexpr int kSampleMaxGrid = 160;                    // CTAs whose candidates one CTA can merge
 
 // ---- weight tape ------------------------------------------------------------
 // The tape is one device buffer. CTA c owns a contiguous region holding, in
@@ -112,8 +114,7 @@ struct Params {
   unsigned long long* fo;     // [hq*dh] attention output
   unsigned long long* fh;     // [hbuf] FFN hidden (dense: ff; MoE: ffs + top_k*ffe)
   unsigned long long* fcand;  // [grid][3] LM-head candidates: best value, its index, second value
-  float* apart;               // attention partials [hq][max_chunks][dh + 4]
-  unsigned int* acnt;         // [L][hk] per-layer, per-KV-head arrival counters (grow within a launch)
+  unsigned long long* apart;  // attention chunk records [hq][max_chunks][dh + 4]: (max, sum), pad, acc[dh]
   Ctrl* ctrl;
   int max_chunks;
   // run
@@ -126,6 +127,14 @@ struct Params {
   int fault_cta, fault_barrier;
   unsigned long long* trace; // device [grid][trace_cap][2] or null
   int trace_cap;
+  // sampling (temperature > 0; greedy otherwise): top-k in [1, kSampleK],
+  // top-p in (0, 1], Philox key `seed`. fsamp holds, flagged like the scratch
+  // above, each CTA's local top-k as (value, index) word pairs [grid][2 *
+  // kSampleK] and then the sampled token's word; cleared before a sampling launch.
+  float samp_temp, samp_p;
+  int samp_k;
+  unsigned long long samp_seed;
+  unsigned long long* fsamp;
   int n_stages;     // multiple of kConsumerWarps: stage s belongs to warp s % kConsumerWarps
   int stage_bytes;
   int vec_floats;   // shared vector buffer, including the norm-gain buffer at gbuf_off

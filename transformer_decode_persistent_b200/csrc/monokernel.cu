@@ -48,7 +48,6 @@ constexpr int kErrDevice = -6;   // KIE_ERR_DEVICE
 
 constexpr int kRouteRing = 8;  // routing decisions kept for lagging issuer lanes
 constexpr int kRopeStage = 128; // RoPE pairs whose coefficients are staged in shared memory
-constexpr int kAttnOneChunk = 2; // up to this many 224-position blocks, a KV head stays in one CTA
 
 struct SmemCtl {
   uint64_t full[kMaxStages];
@@ -62,6 +61,10 @@ struct SmemCtl {
   float red[64];
   float ssq[kConsumerWarps];  // per-warp sums of squares of the last RMSNorm input
   float2 rcs[kRopeStage];     // RoPE (cos, sin) of this CTA's first q/k pairs at this step's position
+  unsigned sel_hist[256];     // sampling: radix-select histogram
+  unsigned long long sel_key[kSampleK];  // sampling: the selected top-k keys, then sorted
+  unsigned long long sel_prefix;
+  int sel_need, sel_count;
   Cand wcand[kConsumerWarps];
   unsigned bcast;
   // this CTA's rows of the residual stream: the output projection and the
@@ -340,6 +343,44 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[N], int lane) {
   return r;
 }
 
+// ---------------------------------------------------------------- sampling helpers
+
+// Philox4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel random numbers: as
+// easy as 1, 2, 3", SC 2011): ten rounds of two 32x32->64-bit products on the
+// counter words, the key bumped by the Weyl constants between rounds. Returns
+// the first output word.
+__device__ __forceinline__ uint32_t philox_w0(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3, uint32_t k0,
+                                              uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
+    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+  }
+  return c0;
+}
+
+// Sampling order key: larger logit first, then lower index. The float maps to
+// an unsigned integer with the same order; the index is stored inverted.
+__device__ __forceinline__ unsigned long long sample_key(float v, int idx) {
+  const unsigned b = __float_as_uint(v);
+  const unsigned o = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  return ((unsigned long long)o << 32) | (0xFFFFFFFFu - (unsigned)idx);
+}
+__device__ __forceinline__ float key_value(unsigned long long k) {
+  const unsigned o = (unsigned)(k >> 32);
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
+}
+__device__ __forceinline__ int key_index(unsigned long long k) { return (int)(0xFFFFFFFFu - (unsigned)k); }
+
 // ---------------------------------------------------------------- errors
 
 __device__ void record_error(const Params& P, int code, int where, int step) {
@@ -393,15 +434,8 @@ __device__ __forceinline__ AttnPlan attn_plan(int pos, int hk, int grid) {
   constexpr int kUnitMin = kConsumerWarps * kAttnSub;
   AttnPlan a;
   a.T = pos + 1;
-  int per;
-  if (a.T <= kAttnOneChunk * kUnitMin) {
-    // short context: each KV head in one CTA, so no cross-CTA merge of
-    // chunk partials (a merge costs two dependent L2 round trips)
-    per = ((a.T + kUnitMin - 1) / kUnitMin) * kUnitMin;
-  } else {
-    per = (int)(((long long)a.T * hk + grid - 1) / grid);
-    per = ((max(per, kUnitMin) + kUnitMin - 1) / kUnitMin) * kUnitMin;
-  }
+  int per = (int)(((long long)a.T * hk + grid - 1) / grid);
+  per = ((max(per, kUnitMin) + kUnitMin - 1) / kUnitMin) * kUnitMin;
   a.per = per;
   a.pw = per / kConsumerWarps;
   a.nsb = a.pw / kAttnSub;
@@ -649,7 +683,6 @@ struct Consumer {
   const int tid, warp, lane;
   unsigned tbase = 0;   // ring position (tiles consumed by the CTA so far)
   unsigned bar_no = 0;  // grid barriers passed
-  unsigned abase = 0;   // attention arrival-counter increments of the earlier steps of this launch
   int step = 0;
   unsigned route_round = 0;
 
@@ -1182,81 +1215,103 @@ struct Consumer {
 #pragma unroll
           for (int e = 0; e < DPL; e += 2) st_flag2(ob + e, a[e] * inv, a[e + 1] * inv, epoch(l));
         } else {
-          float* gb = P.apart + ((size_t)h * P.max_chunks + ch) * WS;
-          if (lane == 0) {
-            gb[0] = M;
-            gb[1] = Ls;
-          }
+          // this chunk's record of head h, flagged: (max, sum) then acc[DH]
+          unsigned long long* gb = P.apart + ((size_t)h * P.max_chunks + ch) * WS;
+          if (lane == 0) st_flag2(gb, M, Ls, epoch(l));
 #pragma unroll
-          for (int e = 0; e < DPL; ++e) gb[4 + lane * DPL + e] = a[e];
-        }
-      }
-      if (ap.nchk > 1) {
-        cbar();
-        if (tid == 0) {
-          unsigned old;
-          asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;"
-                       : "=r"(old)
-                       : "l"(P.acnt + (size_t)l * hk + g)
-                       : "memory");
-          sc->bcast = old;
-        }
-        cbar();
-        // the counters grow through the launch: earlier steps added abase
-        if (sc->bcast == abase + (unsigned)(ap.nchk - 1)) {  // last CTA of this KV head: merge the chunks
-          if (warp < nh) {
-            const int h = h_lo + warp;
-            const int nchk = ap.nchk;
-            const float* hb = P.apart + (size_t)h * P.max_chunks * WS;
-            float M = -INFINITY;
-            for (int c = lane; c < nchk; c += 32) M = fmaxf(M, __ldcg(hb + (size_t)c * WS));
-            M = warp_max(M);
-            float Ls = 0.f, a[DPL];
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) a[e] = 0.f;
-            for (int c0 = 0; c0 < nchk; c0 += 32) {
-              const int nc = min(32, nchk - c0);
-              float wl = 0.f;
-              if (lane < nc) {
-                const float* cb = hb + (size_t)(c0 + lane) * WS;
-                wl = expf(__ldcg(cb) - M);
-                Ls = fmaf(wl, __ldcg(cb + 1), Ls);
-              }
-              for (int cb0 = 0; cb0 < nc; cb0 += 8) {
-                float4 v8[8];
-#pragma unroll
-                for (int uu = 0; uu < 8; ++uu) {
-                  const float* src = hb + (size_t)(c0 + cb0 + uu) * WS + 4 + lane * DPL;
-                  if (cb0 + uu < nc) {
-                    if constexpr (DPL == 4) v8[uu] = __ldcg(reinterpret_cast<const float4*>(src));
-                    else v8[uu] = make_float4(__ldcg(src), __ldcg(src + 1), 0.f, 0.f);
-                  } else {
-                    v8[uu] = make_float4(0.f, 0.f, 0.f, 0.f);
-                  }
-                }
-#pragma unroll
-                for (int uu = 0; uu < 8; ++uu) {
-                  const float w = __shfl_sync(0xffffffffu, wl, (cb0 + uu) & 31);
-                  a[0] = fmaf(w, v8[uu].x, a[0]);
-                  a[1] = fmaf(w, v8[uu].y, a[1]);
-                  if constexpr (DPL == 4) {
-                    a[2] = fmaf(w, v8[uu].z, a[2]);
-                    a[3] = fmaf(w, v8[uu].w, a[3]);
-                  }
-                }
-              }
-            }
-            Ls = warp_sum(Ls);
-            const float inv = 1.0f / Ls;
-            unsigned long long* ob = P.fo + (size_t)h * DH + lane * DPL;
-#pragma unroll
-            for (int e = 0; e < DPL; e += 2) st_flag2(ob + e, a[e] * inv, a[e + 1] * inv, epoch(l));
-          }
+          for (int e = 0; e < DPL; e += 2) st_flag2(gb + 4 + lane * DPL + e, a[e], a[e + 1], epoch(l));
         }
       }
       cbar();  // qs / wp are reused by the next unit
     }
+    // A KV head split into chunks is finished by the CTA of its chunk 0. That
+    // CTA merges only after it has published the records of all its own units,
+    // so no CTA waits for a record that one of its later units would produce.
+    if (ap.nchk > 1) {
+      for (int uo = 0; uo < nu; ++uo) {
+        const int u = blockIdx.x + uo * G;
+        const int g = u / ap.nchk, ch = u - g * ap.nchk;
+        if (ch != 0) continue;
+        const int h_lo = (g * hq + hk - 1) / hk;
+        const int nh = (((g + 1) * hq + hk - 1) / hk) - h_lo;
+        if (warp < nh) merge_chunks<DH>(h_lo + warp, ap.nchk, epoch(l));
+      }
+    }
     tbase += (unsigned)(nu * ap.nsb * kAttnTilesPerRound);
+  }
+
+  // Merge the nchk chunk records of query head h into its attention output, in
+  // chunk order with a running (max, sum, acc) rescaled per chunk. One warp;
+  // lane l owns head dims l*DPL .. l*DPL + DPL - 1. The flagged words of a
+  // batch of chunks are all loaded before any epoch is checked and the stale
+  // ones re-polled together (one L2 round trip once the last chunk is out).
+  template <int DH>
+  __device__ void merge_chunks(int h, int nchk, unsigned ep) {
+    constexpr int DPL = DH / 32, WS = DH + 4, B = 8, NW = 2 + DPL;
+    const unsigned long long* hb = P.apart + (size_t)h * P.max_chunks * WS;
+    float M = -INFINITY, Ls = 0.f, acc[DPL];
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+    for (int c0 = 0; c0 < nchk; c0 += B) {
+      unsigned long long w[B][NW];
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        const unsigned long long* cb = hb + (size_t)(c0 + b) * WS;
+#pragma unroll
+        for (int i = 0; i < NW; ++i) w[b][i] = (unsigned long long)ep << 32;
+        if (c0 + b < nchk) {
+          ld_flag2(cb, w[b][0], w[b][1]);
+#pragma unroll
+          for (int e = 0; e < DPL; e += 2) ld_flag2(cb + 4 + lane * DPL + e, w[b][2 + e], w[b][3 + e]);
+        }
+      }
+      unsigned long long t0 = 0;
+      for (unsigned it = 0;; ++it) {
+        bool stale = false;
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          bool st = false;
+#pragma unroll
+          for (int i = 0; i < NW; ++i) st |= fepoch(w[b][i]) != ep;
+          if (st) {
+            stale = true;
+            const unsigned long long* cb = hb + (size_t)(c0 + b) * WS;
+            ld_flag2(cb, w[b][0], w[b][1]);
+#pragma unroll
+            for (int e = 0; e < DPL; e += 2) ld_flag2(cb + 4 + lane * DPL + e, w[b][2 + e], w[b][3 + e]);
+          }
+        }
+        if (!stale) break;
+        if (it == 0) {
+          t0 = gtimer();
+        } else if ((it & 31) == 0) {
+          if (sc->abort || ld_relaxed(&P.ctrl->abort)) {
+            sc->abort = 1;
+            return;
+          }
+          if (gtimer() - t0 > P.timeout_ns) {
+            record_error(P, kErrTimeout, 6, step);
+            sc->abort = 1;
+            return;
+          }
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        if (c0 + b >= nchk) break;
+        const float m = fval(w[b][0]), l = fval(w[b][1]);
+        const float Mn = fmaxf(M, m);
+        const float so = expf(M - Mn), sn = expf(m - Mn);
+        Ls = Ls * so + l * sn;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[e] = acc[e] * so + fval(w[b][2 + e]) * sn;
+        M = Mn;
+      }
+    }
+    const float inv = 1.0f / Ls;
+    unsigned long long* ob = P.fo + (size_t)h * DH + lane * DPL;
+#pragma unroll
+    for (int e = 0; e < DPL; e += 2) st_flag2(ob + e, acc[e] * inv, acc[e + 1] * inv, ep);
   }
 
   __device__ void attention_dispatch(int l, int pos) {
@@ -1543,7 +1598,6 @@ struct Consumer {
       // before the next step's bulk copies of them (the phases within a step
       // wait on the flagged words they read instead)
       if (!grid_sync()) return;
-      if (ap_nchk(pos) > 1) abase += (unsigned)ap_nchk(pos);
     }
     if (c == 0 && tid == 0) P.ctrl->final_token = tok;
   }
@@ -1554,15 +1608,18 @@ struct Consumer {
     const float inv = norm_scale();
     float v1 = -INFINITY, v2 = -INFINITY;
     int i1 = INT_MAX;
+    const bool sampling = P.samp_temp > 0.f;
     for (int r = tid; r < dl.nrows; r += kConsumerThreads) {
       const float y = row_sum(r, stride) * inv;
       const int row = dl.row0 + r;
       if (P.logits_out) P.logits_out[(size_t)step * P.V + row] = y;
+      if (sampling) vec[r] = (y == y) ? y : -INFINITY;  // the vector buffer is free after the tiles
       cand_merge(v1, i1, v2, y, row, -INFINITY);
     }
     cand_warp_merge(v1, i1, v2);
     if (lane == 0) sc->wcand[warp] = Cand{v1, i1, v2, 0};
     cbar();
+    if (sampling) publish_topk(dl);
     if (tid == 0) {
       float a1 = -INFINITY, a2 = -INFINITY;
       int ai = INT_MAX;
@@ -1572,6 +1629,158 @@ struct Consumer {
       st_flag2(cb, a1, __int_as_float(ai), epoch(P.L));
       st_flag2(cb + 2, a2, 0.f, epoch(P.L));
     }
+  }
+
+  // Sampling, step 1 (every CTA): the CTA's top-k logits by rank (larger
+  // value first, then lower index), published as flagged (value, index) word
+  // pairs in rank order; ranks past the CTA's rows get (-inf, INT_MAX). The
+  // list is padded to an even length, as the reader takes two pairs per load.
+  __device__ void publish_topk(const SegDesc& dl) {
+    const int K = (P.samp_k + 1) & ~1, n = dl.nrows;
+    unsigned long long* dst = P.fsamp + (size_t)blockIdx.x * 2 * kSampleK;
+    const unsigned ep = epoch(P.L);
+    for (int r = tid; r < n; r += kConsumerThreads) {
+      const float y = vec[r];
+      int rank = 0;
+      for (int q = 0; q < n; ++q) {
+        const float z = vec[q];
+        rank += (z > y || (z == y && q < r)) ? 1 : 0;
+      }
+      if (rank < K) st_flag2(dst + 2 * rank, y, __int_as_float(dl.row0 + r), ep);
+    }
+    for (int j = n + tid; j < K; j += kConsumerThreads) st_flag2(dst + 2 * j, -INFINITY, __int_as_float(INT_MAX), ep);
+  }
+
+  // Sampling, step 2 (CTA 0): merge all CTAs' candidates into the global
+  // top-k (radix select of the k-th largest 64-bit order key, 8 bits per
+  // pass), sort them, and pick by the definition of the sampling oracle:
+  // weights exp(z - max z) with z = logit / temperature, the shortest prefix
+  // whose cumulative weight reaches top_p of the total, then the first entry
+  // whose cumulative weight exceeds u times the kept total. u comes from
+  // Philox4x32-10 with counter (position, 0, 0, 0) and key (seed low, seed
+  // high): the top 24 bits of the first word times 2^-24.
+  __device__ int sample_select(int pos) {
+    constexpr int kSlots = (kSampleMaxGrid * kSampleK + kConsumerThreads - 1) / kConsumerThreads;
+    const int K = P.samp_k, n = (int)gridDim.x * K;
+    const unsigned ep = epoch(P.L);
+    unsigned long long key[kSlots];
+#pragma unroll
+    for (int sl = 0; sl < kSlots; ++sl) {
+      const int c = tid + sl * kConsumerThreads;
+      key[sl] = 0ull;
+      if (c < n) {
+        const int cta = c / K, i = c - cta * K;
+        const float4 w = wait4(P.fsamp + (size_t)cta * 2 * kSampleK + 2 * (i & ~1), ep);
+        const bool hi = i & 1;
+        key[sl] = sample_key(hi ? w.z : w.x, __float_as_int(hi ? w.w : w.y));
+      }
+    }
+    unsigned long long prefix = 0ull, pmask = 0ull;
+    int need = K;
+    for (int pass = 0; pass < 8; ++pass) {
+      const int shift = 56 - 8 * pass;
+      for (int b = tid; b < 256; b += kConsumerThreads) sc->sel_hist[b] = 0u;
+      cbar();
+#pragma unroll
+      for (int sl = 0; sl < kSlots; ++sl) {
+        const int c = tid + sl * kConsumerThreads;
+        if (c < n && (key[sl] & pmask) == prefix) atomicAdd(&sc->sel_hist[(key[sl] >> shift) & 255u], 1u);
+      }
+      cbar();
+      if (warp == 0) {
+        // lane l scans bins 255 - 8l down to 248 - 8l; bins are taken from the top
+        unsigned cnt[8], sum = 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          cnt[u] = sc->sel_hist[255 - 8 * lane - u];
+          sum += cnt[u];
+        }
+        unsigned incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        const unsigned excl = incl - sum;
+        if (excl < (unsigned)need && incl >= (unsigned)need) {
+          unsigned acc = excl;
+          int bin = 255 - 8 * lane;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            if (acc + cnt[u] >= (unsigned)need) {
+              bin = 255 - 8 * lane - u;
+              break;
+            }
+            acc += cnt[u];
+          }
+          sc->sel_prefix = prefix | ((unsigned long long)bin << shift);
+          sc->sel_need = need - (int)acc;
+        }
+      }
+      cbar();
+      prefix = sc->sel_prefix;
+      need = sc->sel_need;
+      pmask |= 0xFFull << shift;
+    }
+    // prefix is now the k-th largest key: gather the K keys >= it and sort them
+    if (tid == 0) sc->sel_count = 0;
+    cbar();
+#pragma unroll
+    for (int sl = 0; sl < kSlots; ++sl) {
+      const int c = tid + sl * kConsumerThreads;
+      if (c < n && key[sl] >= prefix) {
+        const int at = atomicAdd(&sc->sel_count, 1);
+        if (at < kSampleK) sc->sel_key[at] = key[sl];
+      }
+    }
+    cbar();
+    unsigned long long mine = 0ull;
+    int rank = 0;
+    if (tid < K) {
+      mine = sc->sel_key[tid];
+      for (int q = 0; q < K; ++q) rank += sc->sel_key[q] > mine ? 1 : 0;
+    }
+    cbar();
+    if (tid < K) sc->sel_key[rank] = mine;
+    cbar();
+    if (warp == 0) {
+      const float invT = 1.0f / P.samp_temp;
+      const unsigned long long ka = lane < K ? sc->sel_key[lane] : 0ull;
+      const unsigned long long kb = lane + 32 < K ? sc->sel_key[lane + 32] : 0ull;
+      const float zmax = __shfl_sync(0xffffffffu, key_value(ka), 0) * invT;
+      const float wa = lane < K ? expf(key_value(ka) * invT - zmax) : 0.f;
+      const float wb = lane + 32 < K ? expf(key_value(kb) * invT - zmax) : 0.f;
+      float ca = wa, cb = wb;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float ta = __shfl_up_sync(0xffffffffu, ca, o), tb = __shfl_up_sync(0xffffffffu, cb, o);
+        if (lane >= o) {
+          ca += ta;
+          cb += tb;
+        }
+      }
+      const float totA = __shfl_sync(0xffffffffu, ca, 31);
+      cb += totA;  // entries lane + 32 follow all of the first 32
+      const float tot = __shfl_sync(0xffffffffu, cb, 31);
+      // cut: the last kept entry
+      int cut = K - 1;
+      if (P.samp_p < 1.f) {
+        const float lim = P.samp_p * tot;
+        const unsigned ma = __ballot_sync(0xffffffffu, lane < K && ca >= lim);
+        const unsigned mb = __ballot_sync(0xffffffffu, lane + 32 < K && cb >= lim);
+        cut = ma ? __ffs(ma) - 1 : (mb ? 32 + __ffs(mb) - 1 : K - 1);
+      }
+      const float kept = cut < 32 ? __shfl_sync(0xffffffffu, ca, cut) : __shfl_sync(0xffffffffu, cb, cut - 32);
+      const uint32_t w0 = philox_w0((uint32_t)pos, 0u, 0u, 0u, (uint32_t)P.samp_seed, (uint32_t)(P.samp_seed >> 32));
+      const float target = (float)(w0 >> 8) * (1.0f / 16777216.0f) * kept;
+      const unsigned pa = __ballot_sync(0xffffffffu, lane <= cut && lane < K && ca > target);
+      const unsigned pb = __ballot_sync(0xffffffffu, lane + 32 <= cut && lane + 32 < K && cb > target);
+      const int pick = pa ? __ffs(pa) - 1 : (pb ? 32 + __ffs(pb) - 1 : cut);
+      const unsigned long long kp = pick < 32 ? __shfl_sync(0xffffffffu, ka, pick) : __shfl_sync(0xffffffffu, kb, pick - 32);
+      if (lane == 0) sc->sel_count = key_index(kp);
+    }
+    cbar();
+    return sc->sel_count;
   }
 
   // Every CTA reduces all CTAs' flagged candidates the same way.
@@ -1593,11 +1802,27 @@ struct Consumer {
       sc->tok = ai;
       sc->margin = a1 - a2;
       if (blockIdx.x == 0) {
-        P.out_tokens[step] = ai;
+        if (P.samp_temp <= 0.f) P.out_tokens[step] = ai;
         if (P.margins_out) P.margins_out[step] = a1 - a2;
       }
     }
     cbar();
+    if (P.samp_temp > 0.f && sc->tok != INT_MAX) {
+      // CTA 0 samples and publishes the token; the others wait for its word
+      unsigned long long* tw = P.fsamp + (size_t)gridDim.x * 2 * kSampleK;
+      if (blockIdx.x == 0) {
+        const int t = sample_select(P.pos0 + step);
+        if (tid == 0) {
+          P.out_tokens[step] = t;
+          st_flag2(tw, __int_as_float(t), 0.f, epoch(P.L));
+          st_flag2(tw + 2, 0.f, 0.f, epoch(P.L));
+          sc->tok = t;
+        }
+      } else if (tid == 0) {
+        sc->tok = __float_as_int(wait4(tw, epoch(P.L)).x);
+      }
+      cbar();
+    }
     return sc->tok;
   }
 };

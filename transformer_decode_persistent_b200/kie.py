@@ -48,7 +48,9 @@ class kie_decode_opts(ctypes.Structure):
     _fields_ = [("forced_tokens", ctypes.c_void_p), ("logits_out", ctypes.c_void_p),
                 ("margins_out", ctypes.c_void_p), ("timeout_ms", ctypes.c_uint32),
                 ("fault_cta", ctypes.c_int32), ("fault_barrier", ctypes.c_int32),
-                ("trace_out", ctypes.c_void_p), ("trace_cap", ctypes.c_int32)]
+                ("trace_out", ctypes.c_void_p), ("trace_cap", ctypes.c_int32),
+                ("temperature", ctypes.c_float), ("top_k", ctypes.c_int32), ("top_p", ctypes.c_float),
+                ("seed", ctypes.c_uint64)]
 
 
 class kie_info(ctypes.Structure):
@@ -247,7 +249,8 @@ class Engine:
 
     def decode(self, n: int, forced=None, logits: bool = False, margins: bool = False,
                out=None, timeout_ms: int = 0, fault: tuple | None = None, trace=None,
-               stream=None):
+               stream=None, temperature: float = 0.0, top_k: int = 0, top_p: float = 1.0,
+               seed: int = 0):
         """Decode n tokens in one launch.
 
         Returns a dict with 'tokens' (numpy int32 [n], or the given ``out``),
@@ -257,10 +260,14 @@ class Engine:
         [grid, cap, 2] for the step barrier's arrival and release times, or,
         on a trace-build engine, [grid, cap, 4] with one record per phase
         (start, input ready, tiles done, epilogue done; records step * (5 L +
-        2) + phase, the step barrier last).
+        2) + phase, the step barrier last). ``temperature`` > 0 samples in the
+        kernel with ``top_k`` (1..64), ``top_p`` and the Philox ``seed``
+        (see kie_decode_opts in include/kie.h); 0 is greedy.
         """
         import torch
-        o = kie_decode_opts(fault_cta=-1, fault_barrier=-1, timeout_ms=int(timeout_ms))
+        o = kie_decode_opts(fault_cta=-1, fault_barrier=-1, timeout_ms=int(timeout_ms),
+                            temperature=float(temperature), top_k=int(top_k), top_p=float(top_p),
+                            seed=int(seed) & 0xFFFFFFFFFFFFFFFF)
         keep = []
         if forced is not None:
             f = np.ascontiguousarray(np.asarray(forced, dtype=np.int32))
