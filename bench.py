@@ -379,6 +379,7 @@ def main():
 
     # end to end through the C ABI with host buffers
     e2e = None
+    prefill = None
     if not args.no_e2e:
         host_out = torch.empty(n, dtype=torch.int32).pin_memory()
         host_prompt = np.ascontiguousarray(prompt.astype(np.int32))
@@ -401,7 +402,19 @@ def main():
         e_ms = max_over_ranks([max(a.elapsed_time(b), wall * 1000.0)])[0]
         e2e = {"value": job_value(n * args.steps, ws, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(host_prompt.nbytes), "d2h_bytes_per_step": int(n * 4),
-               "includes": "reset + prefill of the 256-token prompt from host memory + decode into pinned host memory"}
+               "includes": f"reset + prefill of the {P}-token prompt from host memory + decode into pinned host memory"}
+        # the prompt path alone (tensor-core prefill for dense models)
+        pms = []
+        for _ in range(max(1, args.steps)):
+            eng.reset()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            eng.prefill(host_prompt)
+            b.record(stream)
+            torch.cuda.synchronize()
+            pms.append(a.elapsed_time(b))
+        prefill = {"prompt_tokens": P, "ms": min(pms), "tokens_per_s": (P - 1) / (min(pms) / 1000.0),
+                   "path": "tensor cores" if shape.n_experts == 0 else "decode kernel, forced tokens"}
 
     stall = None
     if args.trace and rank == 0:
@@ -411,9 +424,9 @@ def main():
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         v, steps, dt, threads = cpu_oracle_sample(shape, weights, budget_s=20.0, max_steps=6)
         cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": f"{steps} oracle decode steps of the {shape.name} workload from an empty "
-                         f"context ({dt:.1f} s; per-token cost is the weight GEMVs, attention over "
-                         f"<= {P + n} positions adds < 1%)"}
+               "sample": f"{steps} oracle decode steps (positions 0-{steps - 1}) of the {shape.name} workload "
+                         f"from an empty context on {threads} BLAS threads ({dt:.1f} s; the per-token cost is "
+                         f"the weight GEMVs, attention over <= {P + n} positions adds < 1%)"}
 
     eng.close()
     if rank == 0:
@@ -435,6 +448,7 @@ def main():
                          "frac_of_8TBps_spec": achieved / 8000.0},
             "clocks": clocks,
             "e2e": e2e,
+            "prefill": prefill,
             "cpu_baseline": cpu,
         }
         if stall is not None:

@@ -610,23 +610,13 @@ __device__ __forceinline__ void tile_gemv(uint32_t w_s, uint32_t x_s, uint32_t x
   }
 }
 
-// Tile of g <= GM rows x 32*CPL chunks (rows past g are skipped): the lane's
-// share is copied to registers and the stage released at once, then two
-// accumulators per row, and one butterfly turns the rows' lane partials into
-// lane r holding row r's sum.
+// Tile of g <= GM rows x 32*CPL chunks (rows past g are zeroed): the lane's
+// share is in registers (wr), then two accumulators per row, and one
+// butterfly turns the rows' lane partials into lane r holding row r's sum.
 template <int GM, int CPL>
-__device__ __forceinline__ void tile_gemv_rows(uint32_t w_s, uint32_t x_s, uint32_t xpb, int lane, float* part,
-                                               int pidx0, int pstride, uint64_t* empty, int g) {
-  constexpr int nch = CPL * 32;
+__device__ __forceinline__ void tile_rows_compute(const uint4 (&wr)[GM][CPL], uint32_t x_s, uint32_t xpb, int lane,
+                                                  float* part, int pidx0, int pstride, int g) {
   constexpr int NP = GM <= 8 ? 8 : 16;
-  uint4 wr[GM][CPL];
-#pragma unroll
-  for (int k = 0; k < CPL; ++k)
-#pragma unroll
-    for (int r = 0; r < GM; ++r)
-      wr[r][k] = r < g ? lds_u4(w_s + (uint32_t)(r * nch + lane + 32 * k) * 16u) : make_uint4(0u, 0u, 0u, 0u);
-  __syncwarp();
-  if (lane == 0) mbar_arrive(empty);
   float acc[GM][2];
 #pragma unroll
   for (int r = 0; r < GM; ++r) acc[r][0] = acc[r][1] = 0.f;
@@ -642,6 +632,23 @@ __device__ __forceinline__ void tile_gemv_rows(uint32_t w_s, uint32_t x_s, uint3
   for (int r = 0; r < NP; ++r) v[r] = r < GM ? acc[r][0] + acc[r][1] : 0.f;
   const float t = transpose_reduce<NP>(v, lane);
   if (lane < g) part[pidx0 + lane * pstride] = t;
+}
+
+// The tile from its ring stage: copy the lane's share out and release the
+// stage at once.
+template <int GM, int CPL>
+__device__ __forceinline__ void tile_gemv_rows(uint32_t w_s, uint32_t x_s, uint32_t xpb, int lane, float* part,
+                                               int pidx0, int pstride, uint64_t* empty, int g) {
+  constexpr int nch = CPL * 32;
+  uint4 wr[GM][CPL];
+#pragma unroll
+  for (int k = 0; k < CPL; ++k)
+#pragma unroll
+    for (int r = 0; r < GM; ++r)
+      wr[r][k] = r < g ? lds_u4(w_s + (uint32_t)(r * nch + lane + 32 * k) * 16u) : make_uint4(0u, 0u, 0u, 0u);
+  __syncwarp();
+  if (lane == 0) mbar_arrive(empty);
+  tile_rows_compute<GM, CPL>(wr, x_s, xpb, lane, part, pidx0, pstride, g);
 }
 
 // K/V row slice of one lane (DPL fp16 head dims) from shared memory.
@@ -751,6 +758,8 @@ struct Consumer {
 
   // The flagged words src[i..i+4) for the kLoadBatch groups i = base + b *
   // kConsumerThreads * 4 (those below n), once they carry epoch ep, into v.
+  // Every lane of the warp must call it together (warp-wide votes decide when
+  // the warp stops polling).
   // All of the batch's loads are issued before any epoch is checked, and the
   // groups still stale are re-polled together, so a thread waits about one L2
   // round trip per batch instead of one per group. Bounded: on abort or
@@ -769,6 +778,7 @@ struct Consumer {
       }
     }
     unsigned long long t0 = 0;
+    // the warp loops together (warp-uniform exit and give-up)
     for (unsigned it = 0;; ++it) {
       bool stale = false;
 #pragma unroll
@@ -780,7 +790,7 @@ struct Consumer {
           ld_flag2(src + i + 2, w[b][2], w[b][3]);
         }
       }
-      if (!stale) break;
+      if (!__any_sync(0xffffffffu, stale)) break;
       if (it == 0) {
         t0 = gtimer();
       } else if ((it & 31) == 0) {
@@ -791,7 +801,7 @@ struct Consumer {
           record_error(P, kErrTimeout, 6, step);
           give_up = true;
         }
-        if (give_up) {
+        if (__any_sync(0xffffffffu, give_up)) {
           sc->abort = 1;
 #pragma unroll
           for (int b = 0; b < kLoadBatch; ++b) v[b] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -806,7 +816,10 @@ struct Consumer {
   // vec = the flagged vector src[0..n) of epoch ep (n a multiple of 8), once
   // its producers have written it
   __device__ void load_vec(const unsigned long long* src, unsigned ep, int n) {
-    for (int base = tid * 4; base < n; base += kConsumerThreads * 4 * kLoadBatch) {
+    // warp-uniform trip count: fetch_batch's warp-wide votes need every lane
+    // (lanes past n hold only groups that are already complete)
+    for (int base0 = warp * 128; base0 < n; base0 += kConsumerThreads * 4 * kLoadBatch) {
+      const int base = base0 + lane * 4;
       float4 v[kLoadBatch];
       fetch_batch(src, ep, n, base, v);
 #pragma unroll
@@ -840,7 +853,9 @@ struct Consumer {
     asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's gain copies
     const __half* gb = reinterpret_cast<const __half*>(vec + P.gbuf_off);
     float ss = 0.f;
-    for (int base = tid * 4; base < n; base += kConsumerThreads * 4 * kLoadBatch) {
+    // warp-uniform trip count, as in load_vec
+    for (int base0 = warp * 128; base0 < n; base0 += kConsumerThreads * 4 * kLoadBatch) {
+      const int base = base0 + lane * 4;
       float4 v[kLoadBatch];
       if (srcf) {
         fetch_batch(srcf, ep, n, base, v);
@@ -1854,10 +1869,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       Producer pr(P, sc, ring, lane, dc);
       pr.run();
     }
-    return;
+  } else {
+    Consumer cs(P, sc, part, vec, ring, dc);
+    cs.run();
   }
-  Consumer cs(P, sc, part, vec, ring, dc);
-  cs.run();
 }
 
 // ---- host-side accessors used by the launcher

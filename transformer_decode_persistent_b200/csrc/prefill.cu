@@ -21,8 +21,9 @@
 //  * epilogues: q/k/v (RoPE on adjacent row pairs, q scaled by 1/sqrt(dh), K
 //    and V appended to the fp16 cache the decode kernel reads), residual add
 //    (output and down projections) and SwiGLU (gate/up rows interleaved).
-//  * rmsnorm_split_kernel, embed_kernel and attention_kernel (causal softmax
-//    attention over the cache in fp32 on the CUDA cores).
+//  * rmsnorm_split_kernel, embed_kernel and tc_attention_kernel (causal softmax
+//    attention of the chunk over the cache on the tensor cores, mma.sync with
+//    fp16 hi/lo operands and fp32 accumulators).
 //
 // The last layer's attention, output projection and FFN are skipped: a
 // prompt position contributes nothing but its K and V.
@@ -282,88 +283,232 @@ __global__ void rmsnorm_split_kernel(const float* x, const __half* g, __half* hi
   for (int i = threadIdx.x; i < d; i += blockDim.x) split_store(hi, lo, (size_t)t * d + i, xr[i] * inv * __half2float(g[i]));
 }
 
-// Causal attention of T prompt tokens (positions pos0 .. pos0 + T - 1) over
-// the cache of one layer, in fp32: block (query head h, block of kQB tokens);
-// keys stream through shared memory in blocks of kKB with an online softmax.
-// q is rotated and pre-scaled by 1/sqrt(dh). Output as fp16 hi/lo parts
-// [T][hq * dh] (the next GEMM's operand). 256 threads: 8 threads per query
-// token (kQB = 32), each owning dh / 8 output dims.
-constexpr int kQB = 32, kKB = 32;
+// ---------------------------------------------------------------- tensor-core attention
+//
+// Causal attention of the chunk's queries on the tensor cores (mma.sync
+// m16n8k16, fp16 operands, fp32 accumulators): block (query head h, 64
+// queries), 4 warps of 16 query rows. q (fp32, rotated, pre-scaled) enters as
+// fp16 hi + lo parts held in registers; K and V blocks of 64 keys stream
+// through double-buffered, padded shared memory (cp.async). S = Q_hi K^T +
+// Q_lo K^T; the online softmax runs on the accumulators; P (in [0, 1]) is split
+// into fp16 hi + lo for O += P_hi V + P_lo V, so both products keep about 22
+// bits. Output as fp16 hi/lo parts [T][hq * dh] (the next GEMM's operand).
+constexpr int kTQ = 64, kTK = 64;
 template <int DH>
-__global__ void __launch_bounds__(256) attention_kernel(AttnArgs a) {
-  constexpr int DPT = DH / 8;  // output dims per thread
-  __shared__ float qs[kQB][DH + 1];
-  __shared__ __half ks[kKB][DH + 2];
-  __shared__ __half vs[kKB][DH];
-  __shared__ float ps[kQB][kKB + 1];
+struct TcAttn {
+  static constexpr int LD = DH + 8;  // padded row (halves): ldmatrix rows fall in distinct banks
+  static constexpr int kTileHalves = kTK * LD;
+  static constexpr int kSmem = 2 * 2 * kTileHalves * 2;  // K and V, double-buffered
+};
+
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+  const __half2 h = __floats2half2_rn(a, b);
+  uint32_t u;
+  memcpy(&u, &h, 4);
+  return u;
+}
+__device__ __forceinline__ void split_h2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __half ha = __float2half_rn(a), hb = __float2half_rn(b);
+  const __half2 h = __halves2half2(ha, hb);
+  memcpy(&hi, &h, 4);
+  lo = pack_h2(a - __half2float(ha), b - __half2float(hb));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+template <int DH>
+__global__ void __launch_bounds__(128) tc_attention_kernel(AttnArgs a) {
+  using C = TcAttn<DH>;
+  constexpr int NKS = DH / 16;  // k-steps of q . k
+  constexpr int NDT = DH / 8;   // n-tiles of the output
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  __half* sK = reinterpret_cast<__half*>(smem_raw);  // [2][kTK][LD]
+  __half* sV = sK + 2 * C::kTileHalves;               // [2][kTK][LD]
   const int h = blockIdx.x, qb = blockIdx.y;
   const int g = (h * a.hk) / a.hq;
-  const int qi = threadIdx.x >> 3, sub = threadIdx.x & 7;
-  const int t0 = qb * kQB, t = t0 + qi;
-  const bool live = t < a.T;
-  for (int i = threadIdx.x; i < kQB * DH; i += 256) {
-    const int r = i / DH, c = i - r * DH;
-    qs[r][c] = (t0 + r < a.T) ? a.q[(size_t)(t0 + r) * a.hq * DH + (size_t)h * DH + c] : 0.f;
-  }
-  float m = -INFINITY, l = 0.f, acc[DPT];
-#pragma unroll
-  for (int e = 0; e < DPT; ++e) acc[e] = 0.f;
-  const int last = a.pos0 + min(a.T, t0 + kQB) - 1;  // last key any query of this block sees
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int t0 = qb * kTQ;                      // first query (chunk index) of the block
+  const int rw = t0 + warp * 16;                // first query row of this warp
+  const int qlast = min(a.T, t0 + kTQ) - 1;     // last query of the block
+  const int last = a.pos0 + qlast;              // last key any query of the block sees
   const __half* K = a.kcache + (size_t)(a.layer * a.hk + g) * a.max_ctx * DH;
   const __half* V = a.vcache + (size_t)(a.layer * a.hk + g) * a.max_ctx * DH;
-  for (int j0 = 0; j0 <= last; j0 += kKB) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < kKB * DH / 2; i += 256) {
-      const int r = (2 * i) / DH, c = 2 * i - r * DH;
-      __half2 kv = __floats2half2_rn(0.f, 0.f), vv = kv;
-      if (j0 + r <= last) {
-        kv = *reinterpret_cast<const __half2*>(K + (size_t)(j0 + r) * DH + c);
-        vv = *reinterpret_cast<const __half2*>(V + (size_t)(j0 + r) * DH + c);
-      }
-      *reinterpret_cast<__half2*>(&ks[r][c]) = kv;
-      *reinterpret_cast<__half2*>(&vs[r][c]) = vv;
-    }
-    __syncthreads();
-    // scores: thread (qi, sub) computes keys sub, sub + 8, ... of the block
-    const int pos = a.pos0 + t;
-    float smax = -INFINITY;
-    for (int jj = sub; jj < kKB; jj += 8) {
-      float s = 0.f;
-#pragma unroll 8
-      for (int c = 0; c < DH; ++c) s = fmaf(qs[qi][c], __half2float(ks[jj][c]), s);
-      s = (live && j0 + jj <= pos) ? s : -INFINITY;
-      ps[qi][jj] = s;
-      smax = fmaxf(smax, s);
-    }
+
+  // q fragments (A operand, row-major 16 x 16 per k-step) as hi and lo parts
+  uint32_t qh[NKS][4], ql[NKS][4];
+  {
+    const int r0 = rw + gid, r1 = rw + gid + 8;
+    const float* q0 = a.q + (size_t)r0 * a.hq * DH + (size_t)h * DH;
+    const float* q1 = a.q + (size_t)r1 * a.hq * DH + (size_t)h * DH;
 #pragma unroll
-    for (int o = 4; o > 0; o >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
-    const float mn = fmaxf(m, smax);
-    const float corr = (mn == -INFINITY) ? 1.f : expf(m - mn);
-    float psum = 0.f;
-    for (int jj = sub; jj < kKB; jj += 8) {
-      const float s = ps[qi][jj];
-      const float p = (s == -INFINITY) ? 0.f : expf(s - mn);
-      ps[qi][jj] = p;
-      psum += p;
-    }
-#pragma unroll
-    for (int o = 4; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
-    __syncwarp();
-    l = l * corr + psum;
-    m = mn;
-#pragma unroll
-    for (int e = 0; e < DPT; ++e) acc[e] *= corr;
-    for (int jj = 0; jj < kKB; ++jj) {
-      const float p = ps[qi][jj];
-#pragma unroll
-      for (int e = 0; e < DPT; ++e) acc[e] = fmaf(p, __half2float(vs[jj][sub * DPT + e]), acc[e]);
+    for (int ks = 0; ks < NKS; ++ks) {
+      const int c = ks * 16 + tig * 2;
+      float2 x00 = make_float2(0.f, 0.f), x10 = x00, x01 = x00, x11 = x00;
+      if (r0 < a.T) { x00 = *reinterpret_cast<const float2*>(q0 + c); x01 = *reinterpret_cast<const float2*>(q0 + c + 8); }
+      if (r1 < a.T) { x10 = *reinterpret_cast<const float2*>(q1 + c); x11 = *reinterpret_cast<const float2*>(q1 + c + 8); }
+      split_h2(x00.x, x00.y, qh[ks][0], ql[ks][0]);
+      split_h2(x10.x, x10.y, qh[ks][1], ql[ks][1]);
+      split_h2(x01.x, x01.y, qh[ks][2], ql[ks][2]);
+      split_h2(x11.x, x11.y, qh[ks][3], ql[ks][3]);
     }
   }
-  if (live) {
-    const float inv = 1.0f / l;
-    const size_t base = (size_t)t * a.hq * DH + (size_t)h * DH + sub * DPT;
+  float o[NDT][4];
 #pragma unroll
-    for (int e = 0; e < DPT; ++e) split_store(a.o_hi, a.o_lo, base + e, acc[e] * inv);
+  for (int i = 0; i < NDT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // rows gid and gid + 8
+  const int pos_r0 = a.pos0 + rw + gid, pos_r1 = pos_r0 + 8;
+
+  // K/V block loader: 64 rows x DH halves each, 16-byte cp.async pieces
+  auto load_kv = [&](int buf, int j0) {
+    constexpr int PIECES = kTK * DH / 8;
+    __half* dk = sK + buf * C::kTileHalves;
+    __half* dv = sV + buf * C::kTileHalves;
+    for (int i = threadIdx.x; i < PIECES; i += 128) {
+      const int r = i / (DH / 8), c = (i - r * (DH / 8)) * 8;
+      const int key = min(j0 + r, last);  // rows past `last` repeat a valid row (masked below)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(su32(dk + r * C::LD + c)),
+                   "l"(K + (size_t)key * DH + c)
+                   : "memory");
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(su32(dv + r * C::LD + c)),
+                   "l"(V + (size_t)key * DH + c)
+                   : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  const int nkb = last / kTK + 1;
+  load_kv(0, 0);
+  for (int kb = 0; kb < nkb; ++kb) {
+    const int buf = kb & 1;
+    if (kb + 1 < nkb) {
+      load_kv(buf ^ 1, (kb + 1) * kTK);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncthreads();
+    const int j0 = kb * kTK;
+    const __half* cK = sK + buf * C::kTileHalves;
+    const __half* cV = sV + buf * C::kTileHalves;
+    // S = Q K^T for 16 rows x 64 keys: 8 n-tiles of 8 keys
+    float s[kTK / 8][4];
+#pragma unroll
+    for (int nt = 0; nt < kTK / 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < NKS; ++ks) {
+#pragma unroll
+      for (int np = 0; np < kTK / 16; ++np) {
+        // B fragments of two n-tiles (keys 16np .. 16np + 15) for dims 16ks .. 16ks + 15:
+        // matrices (keys +0..7, dims +0..7), (+0..7, +8..15), (+8..15, +0..7), (+8..15, +8..15)
+        const int mi = lane >> 3, mr = lane & 7;
+        const int key = np * 16 + (mi >> 1) * 8 + mr, dim = ks * 16 + (mi & 1) * 8;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(su32(cK + key * C::LD + dim), b0, b1, b2, b3);
+        mma16816(s[2 * np], qh[ks], b0, b1);
+        mma16816(s[2 * np], ql[ks], b0, b1);
+        mma16816(s[2 * np + 1], qh[ks], b2, b3);
+        mma16816(s[2 * np + 1], ql[ks], b2, b3);
+      }
+    }
+    // causal mask and online softmax (rows gid, gid + 8; each row over the quad)
+    float mx0 = m0, mx1 = m1;
+#pragma unroll
+    for (int nt = 0; nt < kTK / 8; ++nt) {
+      const int k0 = j0 + nt * 8 + tig * 2;
+      if (k0 > pos_r0) s[nt][0] = -INFINITY;
+      if (k0 + 1 > pos_r0) s[nt][1] = -INFINITY;
+      if (k0 > pos_r1) s[nt][2] = -INFINITY;
+      if (k0 + 1 > pos_r1) s[nt][3] = -INFINITY;
+      mx0 = fmaxf(mx0, fmaxf(s[nt][0], s[nt][1]));
+      mx1 = fmaxf(mx1, fmaxf(s[nt][2], s[nt][3]));
+    }
+#pragma unroll
+    for (int o2 = 1; o2 < 4; o2 <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o2));
+    }
+    const float c0 = (mx0 == -INFINITY) ? 1.f : expf(m0 - mx0);
+    const float c1 = (mx1 == -INFINITY) ? 1.f : expf(m1 - mx1);
+    float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < kTK / 8; ++nt) {
+      s[nt][0] = (s[nt][0] == -INFINITY) ? 0.f : expf(s[nt][0] - mx0);
+      s[nt][1] = (s[nt][1] == -INFINITY) ? 0.f : expf(s[nt][1] - mx0);
+      s[nt][2] = (s[nt][2] == -INFINITY) ? 0.f : expf(s[nt][2] - mx1);
+      s[nt][3] = (s[nt][3] == -INFINITY) ? 0.f : expf(s[nt][3] - mx1);
+      ps0 += s[nt][0] + s[nt][1];
+      ps1 += s[nt][2] + s[nt][3];
+    }
+#pragma unroll
+    for (int o2 = 1; o2 < 4; o2 <<= 1) {
+      ps0 += __shfl_xor_sync(0xffffffffu, ps0, o2);
+      ps1 += __shfl_xor_sync(0xffffffffu, ps1, o2);
+    }
+    l0 = l0 * c0 + ps0;
+    l1 = l1 * c1 + ps1;
+    m0 = mx0;
+    m1 = mx1;
+#pragma unroll
+    for (int i = 0; i < NDT; ++i) {
+      o[i][0] *= c0;
+      o[i][1] *= c0;
+      o[i][2] *= c1;
+      o[i][3] *= c1;
+    }
+    // O += P V: P from the S accumulators (A layout), V via transposed ldmatrix
+#pragma unroll
+    for (int kk = 0; kk < kTK / 16; ++kk) {
+      uint32_t ph[4], pl[4];
+      split_h2(s[2 * kk][0], s[2 * kk][1], ph[0], pl[0]);
+      split_h2(s[2 * kk][2], s[2 * kk][3], ph[1], pl[1]);
+      split_h2(s[2 * kk + 1][0], s[2 * kk + 1][1], ph[2], pl[2]);
+      split_h2(s[2 * kk + 1][2], s[2 * kk + 1][3], ph[3], pl[3]);
+#pragma unroll
+      for (int dp = 0; dp < NDT / 2; ++dp) {
+        // B fragments of two dim n-tiles (dims 16dp .. 16dp + 15) for keys 16kk .. 16kk + 15:
+        // transposed matrices (keys +0..7, dims +0..7), (+8..15, +0..7), (+0..7, +8..15), (+8..15, +8..15)
+        const int mi = lane >> 3, mr = lane & 7;
+        const int key = kk * 16 + (mi & 1) * 8 + mr, dim = dp * 16 + (mi >> 1) * 8;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(su32(cV + key * C::LD + dim), b0, b1, b2, b3);
+        mma16816(o[2 * dp], ph, b0, b1);
+        mma16816(o[2 * dp], pl, b0, b1);
+        mma16816(o[2 * dp + 1], ph, b2, b3);
+        mma16816(o[2 * dp + 1], pl, b2, b3);
+      }
+    }
+    __syncthreads();  // this buffer is reloaded two blocks on
+  }
+  // O / l to the fp16 hi/lo output
+  const int r0 = rw + gid, r1 = r0 + 8;
+  const float i0 = 1.0f / l0, i1 = 1.0f / l1;
+#pragma unroll
+  for (int nt = 0; nt < NDT; ++nt) {
+    const int c = nt * 8 + tig * 2;
+    if (r0 < a.T) {
+      const size_t at = (size_t)r0 * a.hq * DH + (size_t)h * DH + c;
+      split_store(a.o_hi, a.o_lo, at, o[nt][0] * i0);
+      split_store(a.o_hi, a.o_lo, at + 1, o[nt][1] * i0);
+    }
+    if (r1 < a.T) {
+      const size_t at = (size_t)r1 * a.hq * DH + (size_t)h * DH + c;
+      split_store(a.o_hi, a.o_lo, at, o[nt][2] * i1);
+      split_store(a.o_hi, a.o_lo, at + 1, o[nt][3] * i1);
+    }
   }
 }
 
@@ -427,11 +572,24 @@ cudaError_t rmsnorm_split(const float* x, const __half* g, __half* hi, __half* l
 }
 
 cudaError_t attention(const AttnArgs& a, cudaStream_t st) {
-  const dim3 grid(a.hq, (a.T + kQB - 1) / kQB);
-  if (a.dh == 128) attention_kernel<128><<<grid, 256, 0, st>>>(a);
-  else attention_kernel<64><<<grid, 256, 0, st>>>(a);
+  const dim3 grid(a.hq, (a.T + kTQ - 1) / kTQ);
+  static bool attr[64][2] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int k = a.dh == 128 ? 1 : 0;
+  if (dev < 0 || dev >= 64 || !attr[dev][k]) {
+    cudaError_t e = k ? cudaFuncSetAttribute(tc_attention_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             TcAttn<128>::kSmem)
+                      : cudaFuncSetAttribute(tc_attention_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             TcAttn<64>::kSmem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr[dev][k] = true;
+  }
+  if (k) tc_attention_kernel<128><<<grid, 128, TcAttn<128>::kSmem, st>>>(a);
+  else tc_attention_kernel<64><<<grid, 128, TcAttn<64>::kSmem, st>>>(a);
   return cudaGetLastError();
 }
+
 
 }  // namespace pf
 }  // namespace kie

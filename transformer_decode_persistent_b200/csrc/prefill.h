@@ -53,6 +53,7 @@ cudaError_t gemm(const CUtensorMap& A, const CUtensorMap& Bh, const CUtensorMap&
 cudaError_t embed(const int* tok, const __half* E, float* x, int T, int d, cudaStream_t st);
 cudaError_t rmsnorm_split(const float* x, const __half* g, __half* hi, __half* lo, int T, int d, float eps,
                           cudaStream_t st);
+// causal attention of a chunk over the cache on the tensor cores (mma.sync)
 cudaError_t attention(const AttnArgs& a, cudaStream_t st);
 
 }  // namespace pf
