@@ -59,13 +59,15 @@ typedef enum {
  * of 8; head_dim 64 or 128; each KV head serves 1 to 4 query heads (query
  * head h reads KV head floor(h * n_kv_heads / n_heads)); max_ctx >= 1.
  * Capacity of one launch (one CTA per SM, S SMs): the rows of every matrix are
- * split over the CTAs, and a CTA keeps at most 64 residual rows (d_model <=
- * 64 S, checked by kie_create) and at most 1280 partial sums per phase (its
- * rows of the matrix times the matrix's column blocks of 512 or 768 inputs).
- * With S = 148 and d_model = 2560 (5 column blocks) that bounds the vocabulary
- * at 37,888 and the gate/up width at 18,944 (2 ffn rows of 5 blocks each per
- * unit). kie_load_weights and kie_plan reject a shape past these bounds with
- * KIE_ERR_INVALID_ARG ("a CTA would hold N partial sums (max 1280)"). */
+ * split over the CTAs; a CTA keeps at most 64 residual rows (d_model <= 64 S,
+ * checked by kie_create) and at most 1280 partial sums per phase (its rows of
+ * the matrix times the matrix's column blocks of 512 or 768 inputs). The LM
+ * head and the dense gate/up projection run in row chunks, so any vocabulary
+ * and FFN width fit; the q/k/v, output and down projections and the MoE
+ * phases must fit whole (at S = 148: down projection width up to about
+ * 15,000). MoE: up to 256 experts, top_k up to 8. kie_load_weights and
+ * kie_plan reject a shape past these bounds with KIE_ERR_INVALID_ARG ("a CTA
+ * would hold N partial sums (max 1280)"). */
 typedef struct {
   int32_t n_layers, d_model, n_heads, n_kv_heads, head_dim, ffn, vocab;
   int32_t n_experts, top_k, ffn_expert, ffn_shared;

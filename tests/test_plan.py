@@ -97,12 +97,17 @@ def test_plan_invariants(shape, grid, stage):
         off += int(e["nrows"]) * sh["lm_head"]["K"] * 2
     assert off == info["tape_bytes"]
 
-    # partial sums per phase fit the kernel's buffer (dense phases)
+    # partial sums per phase fit the kernel's buffer (dense phases); gate/up
+    # and the LM head run in row chunks, so one tile group has to fit
     if not shape.n_experts:
         for l in range(L):
             for s_, kind in enumerate(kinds):
-                assert (r[:, l * slots + s_]["nrows"] * sh[kind]["nk"] <= PART_FLOATS).all()
-        assert (r[:, L * slots]["nrows"] * sh["lm_head"]["nk"] <= PART_FLOATS).all()
+                n = r[:, l * slots + s_]["nrows"]
+                if kind == "gate_up":
+                    n = np.minimum(n, sh[kind]["g"])
+                assert (n * sh[kind]["nk"] <= PART_FLOATS).all()
+        n = np.minimum(r[:, L * slots]["nrows"], sh["lm_head"]["g"])
+        assert (n * sh["lm_head"]["nk"] <= PART_FLOATS).all()
 
 
 def test_plan_tape_is_the_weight_bytes():
@@ -143,10 +148,16 @@ def test_plan_rejects_shapes_like_create():
 
 
 def test_plan_rejects_more_partial_sums_than_the_kernel_holds():
-    """32000 LM-head rows over 16 CTAs are 2000 rows per CTA: with any column
-    split that is more partial sums than one CTA holds."""
+    """The LM head runs in row chunks, so 32000 rows over 16 CTAs (2000 rows
+    per CTA) plan fine; a down projection is not chunked, and 64 rows per CTA
+    of a 30720-wide one (40 column blocks of 768) are more partial sums than
+    one CTA holds."""
+    info, _ = K.plan(S.SMALL, 16, 13312)
+    assert info["shapes"]["lm_head"]["g"] * info["shapes"]["lm_head"]["nk"] <= 1280
+    wide = S.Shape("wide-down", n_layers=1, d_model=1024, n_heads=8, n_kv_heads=8, head_dim=128,
+                   ffn=30720, vocab=1000, max_ctx=16)
     with pytest.raises(K.KieError) as ei:
-        K.plan(S.SMALL, 16, 13312)
+        K.plan(wide, 16, 13312)
     assert ei.value.status == -1 and "partial sums" in str(ei.value)
 
 

@@ -65,6 +65,8 @@ struct kie_ctx {
   float2* rope = nullptr;
   unsigned long long* fsamp = nullptr;  // sampling candidates (allocated on first use)
   size_t fsamp_bytes = 0;
+  float* lm_logits = nullptr;           // sampling: per-CTA LM-head logits of a step
+  int lm_rows = 0;                      // most LM-head rows of one CTA
   // Ctrl | flagged scratch (fx, fq, fo, fh, fcand, attention chunk records), cleared before every launch
   unsigned char* syncblk = nullptr;
   size_t syncblk_bytes = 0;
@@ -346,7 +348,8 @@ kie_status make_plan(kie_ctx* c, const kie_config& k, int G, int sb, Plan& plan)
         worst = std::max(worst, Dl[0].nrows * shp[SK_QKV].nk);
         worst = std::max(worst, Dl[1].nrows * shp[SK_O].nk);
         if (!moe) {
-          worst = std::max(worst, Dl[2].nrows * shp[SK_GU].nk);
+          // gate/up runs in row chunks: one tile group of partial sums must fit
+          worst = std::max(worst, std::min(Dl[2].nrows, shp[SK_GU].g) * shp[SK_GU].nk);
           worst = std::max(worst, Dl[3].nrows * shp[SK_DOWN].nk);
         } else {
           int eg = 0;
@@ -355,7 +358,8 @@ kie_status make_plan(kie_ctx* c, const kie_config& k, int G, int sb, Plan& plan)
           worst = std::max(worst, Dl[3].nrows * (shp[SK_SDOWN].nk + k.top_k * shp[SK_EDOWN].nk));
         }
       }
-      worst = std::max(worst, D[(size_t)L * slots].nrows * shp[SK_LM].nk);
+      // the LM head runs in row chunks too
+      worst = std::max(worst, std::min(D[(size_t)L * slots].nrows, shp[SK_LM].g) * shp[SK_LM].nk);
     }
     if (worst > kPartFloats)
       return fail(c, KIE_ERR_INVALID_ARG, "a CTA would hold %d partial sums (max %d)", worst, kPartFloats);
@@ -839,6 +843,9 @@ kie_status kie_load_weights(kie_ctx* c, const kie_tensor* tensors, int n, void* 
     return s;
   }
   for (int i = 0; i < SK_COUNT; ++i) c->shp[i] = plan.shp[i];
+  c->lm_rows = 0;
+  for (int ci = 0; ci < G; ++ci)
+    c->lm_rows = std::max(c->lm_rows, plan.desc[(size_t)ci * (L * c->slots + 1) + (size_t)L * c->slots].nrows);
   auto kind_of = [&](int l, int slot) -> int { return ::kind_of(k, l, slot); };
   const int per_cta = L * c->slots + 1;
   const std::vector<SegDesc>& desc = plan.desc;
@@ -1059,6 +1066,8 @@ Params make_params(const kie_ctx* c, const Run& r, unsigned char* sync_base) {
   P.gbuf_off = c->gbuf_off;
   P.samp_temp = r.temperature; P.samp_p = r.top_p; P.samp_k = r.top_k; P.samp_seed = r.seed;
   P.fsamp = c->fsamp;
+  P.lm_logits = c->lm_logits;
+  P.lm_rows = c->lm_rows;
   return P;
 }
 
@@ -1187,6 +1196,10 @@ kie_status kie_decode(kie_ctx* c, int n, int32_t* out_tokens, const kie_decode_o
     if (!c->fsamp) {
       c->fsamp_bytes = ((size_t)c->grid * 2 * kSampleK + 4) * 8;
       kie_status s0 = dalloc(c, &c->fsamp, c->fsamp_bytes);
+      if (s0) return s0;
+    }
+    if (!c->lm_logits) {
+      kie_status s0 = dalloc(c, &c->lm_logits, (size_t)c->grid * std::max(1, c->lm_rows) * 4);
       if (s0) return s0;
     }
   }

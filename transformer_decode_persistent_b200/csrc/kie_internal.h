@@ -20,9 +20,9 @@ constexpr int kMaxRowsPerTile = 8;                     // rows of one tile in ge
 constexpr int kMaxRowsWide = 13;                       // rows of a tile 512 halves wide
 constexpr int kPartFloats = 1280;                      // per-CTA partial-sum slots per phase
 constexpr int kMaxHeadsPerGroup = 4;                   // query heads per KV head (GQA)
-constexpr int kMaxTopK = 4;                            // routed experts per token
+constexpr int kMaxTopK = 8;                            // routed experts per token
 constexpr int kAttnSub = 32;                           // positions per attention sub-block
-constexpr int kMaxExperts = 64;
+constexpr int kMaxExperts = 256;
 constexpr int kMaxOwnRows = 64;                        // residual rows a CTA keeps in shared memory
 constexpr int kSampleK = 64;                           // largest top-k of in-kernel sampling
 constexpr int kSampleMaxGrid = 160;                    // CTAs whose candidates one CTA can merge
@@ -135,6 +135,8 @@ struct Params {
   int samp_k;
   unsigned long long samp_seed;
   unsigned long long* fsamp;
+  float* lm_logits;           // sampling: this step's LM-head logits of each CTA's rows [grid][lm_rows]
+  int lm_rows;
   int n_stages;     // multiple of kConsumerWarps: stage s belongs to warp s % kConsumerWarps
   int stage_bytes;
   int vec_floats;   // shared vector buffer, including the norm-gain buffer at gbuf_off

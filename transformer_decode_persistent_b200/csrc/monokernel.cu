@@ -1437,30 +1437,48 @@ struct Consumer {
       if (lane == 0) part[e] = a * norm_scale();
     }
     cbar();
-    if (tid == 0) {
+    if (warp == 0) {
+      // top_k rounds of a warp arg-max over the softmax numerators (the
+      // denominator cancels in the renormalisation), larger first and the
+      // lower expert index on ties; a chosen expert is struck out with -1
+      float* pr = part + kMaxExperts;
       float mx = -INFINITY;
-      for (int e = 0; e < P.E; ++e) mx = fmaxf(mx, part[e]);
-      float* pr = part + kMaxExperts;  // softmax numerators (the denominator cancels below)
-      for (int e = 0; e < P.E; ++e) pr[e] = expf(part[e] - mx);
-      unsigned long long used = 0ull;
-      float wsum = 0.f;
+      for (int e = lane; e < P.E; e += 32) mx = fmaxf(mx, part[e]);
+      mx = warp_max(mx);
+      for (int e = lane; e < P.E; e += 32) pr[e] = expf(part[e] - mx);
+      __syncwarp();
       int* re = sc->route_e[route_round % kRouteRing];
+      float wsum = 0.f;
       for (int k = 0; k < P.top_k; ++k) {
-        int bi = -1;
-        float bv = -INFINITY;
-        for (int e = 0; e < P.E; ++e)
-          if (!((used >> e) & 1ull) && (bi < 0 || pr[e] > bv)) {
-            bi = e;
+        float bv = -1.f;
+        int bi = INT_MAX;
+        for (int e = lane; e < P.E; e += 32)
+          if (pr[e] > bv) {
             bv = pr[e];
+            bi = e;
           }
-        used |= 1ull << bi;
-        re[k] = bi;
-        sc->route_w[k] = bv;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+          if (ov > bv || (ov == bv && oi < bi)) {
+            bv = ov;
+            bi = oi;
+          }
+        }
+        if (lane == 0) {
+          re[k] = bi;
+          sc->route_w[k] = bv;
+          pr[bi] = -1.f;
+        }
         wsum += bv;
+        __syncwarp();
       }
-      for (int k = 0; k < P.top_k; ++k) sc->route_w[k] /= wsum;
-      __threadfence_block();
-      sc->route_seq = route_round + 1;  // hand the choice to the producer lanes
+      if (lane == 0) {
+        for (int k = 0; k < P.top_k; ++k) sc->route_w[k] /= wsum;
+        __threadfence_block();
+        sc->route_seq = route_round + 1;  // hand the choice to the producer lanes
+      }
     }
     cbar();
     ++route_round;
@@ -1534,6 +1552,27 @@ struct Consumer {
         // ---- 2. tiles
         if (kind == PH_ATTN) {
           attention_dispatch(l, pos);
+        } else if (kind == PH_LM || (kind == PH_UP && !P.E)) {
+          // the LM head and the dense gate/up run in row chunks that fit the
+          // partial-sum buffer, each chunk followed by its epilogue (the
+          // chunks are whole tile groups: contiguous in the tape and in the
+          // producer's tile order)
+          const SegDesc& full = kind == PH_LM ? dc.at(P.L, 0) : dc.at(l, 2);
+          const SegShape& sh = P.shp[kind == PH_LM ? SK_LM : SK_GU];
+          const int crows = max(sh.g, (kPartFloats / sh.nk) / sh.g * sh.g);
+          const float inv = norm_scale();
+          float v1 = -INFINITY, v2 = -INFINITY;
+          int i1 = INT_MAX;
+          for (int r0 = 0; r0 < full.nrows; r0 += crows) {
+            const SegDesc sub{full.off + (unsigned long long)r0 * sh.K * 2, full.row0 + r0,
+                              min(crows, full.nrows - r0)};
+            run_segment(sub, sh, vec, 0, sh.nk, 0);
+            cbar();
+            if (kind == PH_LM) epi_lm_rows(sub, r0, inv, v1, i1, v2);
+            else epi_swiglu(sub, 0, sh.nk, 0, 1.0f, epoch(l));
+            cbar();  // the partial sums are reused by the next chunk
+          }
+          if (kind == PH_LM) lm_candidates(full, v1, i1, v2);
         } else {
           const int nseg = (P.E && (kind == PH_UP || kind == PH_DOWN)) ? 1 + P.top_k : 1;
           int pnext = 0;
@@ -1575,9 +1614,7 @@ struct Consumer {
             epi_residual(dc.at(l, 1), P.shp[SK_O].nk, l == 0 ? erow : nullptr, 0, epoch(l));
             break;
           case PH_UP:
-            if (!P.E) {
-              epi_swiglu(dc.at(l, 2), 0, P.shp[SK_GU].nk, 0, 1.0f, epoch(l));
-            } else {
+            if (P.E) {
               epi_swiglu(dc.at(l, 2), 0, P.shp[SK_SGU].nk, 0, 1.0f, epoch(l));
               for (int k = 0; k < P.top_k; ++k)
                 epi_swiglu(dc.at(l, 4 + re[k]), rpb[k], P.shp[SK_EGU].nk, P.ffs + k * P.ffe, rw[k], epoch(l));
@@ -1587,8 +1624,7 @@ struct Consumer {
             epi_residual(dc.at(l, 3), P.E ? P.shp[SK_SDOWN].nk + P.top_k * P.shp[SK_EDOWN].nk : P.shp[SK_DOWN].nk,
                          nullptr, 1, epoch(l));
             break;
-          case PH_LM:
-            epi_lm(dc.at(P.L, 0));
+          case PH_LM:  // run with the tiles, chunk by chunk
             break;
           default:
             break;
@@ -1617,24 +1653,28 @@ struct Consumer {
     if (c == 0 && tid == 0) P.ctrl->final_token = tok;
   }
 
-  // LM-head epilogue: logits (optional copy out) and this CTA's greedy candidate.
-  __device__ void epi_lm(const SegDesc& dl) {
+  // LM-head epilogue of one row chunk (rows r0 .. of this CTA's LM rows):
+  // logits (optional copy out, and kept for sampling) and the thread's
+  // running greedy candidate.
+  __device__ void epi_lm_rows(const SegDesc& sub, int r0, float inv, float& v1, int& i1, float& v2) {
     const int stride = P.shp[SK_LM].nk;
-    const float inv = norm_scale();
-    float v1 = -INFINITY, v2 = -INFINITY;
-    int i1 = INT_MAX;
     const bool sampling = P.samp_temp > 0.f;
-    for (int r = tid; r < dl.nrows; r += kConsumerThreads) {
+    float* keep = sampling ? P.lm_logits + (size_t)blockIdx.x * P.lm_rows + r0 : nullptr;
+    for (int r = tid; r < sub.nrows; r += kConsumerThreads) {
       const float y = row_sum(r, stride) * inv;
-      const int row = dl.row0 + r;
+      const int row = sub.row0 + r;
       if (P.logits_out) P.logits_out[(size_t)step * P.V + row] = y;
-      if (sampling) vec[r] = (y == y) ? y : -INFINITY;  // the vector buffer is free after the tiles
+      if (sampling) keep[r] = (y == y) ? y : -INFINITY;
       cand_merge(v1, i1, v2, y, row, -INFINITY);
     }
+  }
+
+  // This CTA's greedy candidate (value, lowest index, runner-up) published
+  // flagged; with sampling also its local top-k.
+  __device__ void lm_candidates(const SegDesc& dl, float v1, int i1, float v2) {
     cand_warp_merge(v1, i1, v2);
     if (lane == 0) sc->wcand[warp] = Cand{v1, i1, v2, 0};
     cbar();
-    if (sampling) publish_topk(dl);
     if (tid == 0) {
       float a1 = -INFINITY, a2 = -INFINITY;
       int ai = INT_MAX;
@@ -1644,6 +1684,7 @@ struct Consumer {
       st_flag2(cb, a1, __int_as_float(ai), epoch(P.L));
       st_flag2(cb + 2, a2, 0.f, epoch(P.L));
     }
+    if (P.samp_temp > 0.f) publish_topk(dl);
   }
 
   // Sampling, step 1 (every CTA): the CTA's top-k logits by rank (larger
@@ -1654,11 +1695,12 @@ struct Consumer {
     const int K = (P.samp_k + 1) & ~1, n = dl.nrows;
     unsigned long long* dst = P.fsamp + (size_t)blockIdx.x * 2 * kSampleK;
     const unsigned ep = epoch(P.L);
+    const float* y_of = P.lm_logits + (size_t)blockIdx.x * P.lm_rows;
     for (int r = tid; r < n; r += kConsumerThreads) {
-      const float y = vec[r];
+      const float y = y_of[r];
       int rank = 0;
       for (int q = 0; q < n; ++q) {
-        const float z = vec[q];
+        const float z = y_of[q];
         rank += (z > y || (z == y && q < r)) ? 1 : 0;
       }
       if (rank < K) st_flag2(dst + 2 * rank, y, __int_as_float(dl.row0 + r), ep);
