@@ -65,7 +65,11 @@ typedef enum {
  * head and the dense gate/up projection run in row chunks, so any vocabulary
  * and FFN width fit; the q/k/v, output and down projections and the MoE
  * phases must fit whole (at S = 148: down projection width up to about
- * 15,000). MoE: up to 256 experts, top_k up to 8. kie_load_weights and
+ * 15,000). Each phase's whole input vector (the largest of d_model, n_heads *
+ * head_dim and the FFN width; MoE: ffn_shared + top_k * ffn_expert) is held in
+ * shared memory as fp32 beside the weight ring: about 40,000 values at most
+ * (kie_create: "shape needs too much shared memory"). MoE: up to 256
+ * experts, top_k up to 8. kie_load_weights and
  * kie_plan reject a shape past these bounds with KIE_ERR_INVALID_ARG ("a CTA
  * would hold N partial sums (max 1280)"). */
 typedef struct {

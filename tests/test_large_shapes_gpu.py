@@ -1,6 +1,7 @@
 """Shapes past the per-CTA partial-sum buffer and larger MoE routing, against
-the oracle through the C ABI: a 128,000-token vocabulary and a 49,152-wide
-FFN (the LM head and gate/up run in row chunks), greedy and sampled; and 128
+the oracle through the C ABI: a 128,000-token vocabulary and a gate/up
+projection of 2 x 24,576 rows over 2,048 inputs (both run in row chunks; 3,460
+and 1,336 partial sums per CTA against 1,280), greedy and sampled; and 128
 routed experts with top-8."""
 import numpy as np
 import pytest
@@ -12,8 +13,8 @@ from parity import check_step_logits, check_tokens, forced_sequence_case, logit_
 
 pytestmark = pytest.mark.gpu
 
-WIDE = S.Shape("wide-vocab-ffn", n_layers=2, d_model=1024, n_heads=8, n_kv_heads=8, head_dim=128,
-               ffn=49152, vocab=128000, prompt_len=16, decode_len=12, max_ctx=48)
+WIDE = S.Shape("wide-vocab-ffn", n_layers=1, d_model=2048, n_heads=16, n_kv_heads=8, head_dim=128,
+               ffn=24576, vocab=128000, prompt_len=16, decode_len=12, max_ctx=48)
 MOE_WIDE = S.Shape("moe-128x-top8", n_layers=2, d_model=512, n_heads=8, n_kv_heads=2, head_dim=64,
                    ffn=0, vocab=3000, n_experts=128, top_k=8, ffn_expert=64, ffn_shared=256,
                    prompt_len=20, decode_len=24, max_ctx=48)
@@ -30,8 +31,8 @@ def wide():
 def test_chunked_lm_head_and_gate_up(wide):
     w, eng = wide
     gl, ol, gt, gm = forced_sequence_case(WIDE, 31, WIDE.decode_len, weights=w, engine=eng)
-    check_step_logits(gl, ol, "128K vocabulary, 49K FFN")
-    check_tokens(gt, ol, "128K vocabulary, 49K FFN")
+    check_step_logits(gl, ol, "128K vocabulary, chunked gate/up")
+    check_tokens(gt, ol, "128K vocabulary, chunked gate/up")
     srt = np.sort(gl, axis=-1)
     assert np.array_equal(gm, srt[:, -1] - srt[:, -2])
 

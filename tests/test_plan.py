@@ -16,7 +16,7 @@ GQA_ODD = S.Shape("gqa-odd", n_layers=3, d_model=512, n_heads=10, n_kv_heads=8, 
 MOE_SMALL = S.Shape("moe-small", n_layers=2, d_model=512, n_heads=8, n_kv_heads=2, head_dim=64, ffn=0,
                     vocab=3000, n_experts=6, top_k=2, ffn_expert=352, ffn_shared=704, max_ctx=64)
 SHAPES = [S.TINY, S.SMALL, S.DENSE_2B, S.LONG_2B, S.MOE, GQA_ODD, MOE_SMALL]
-GEOMETRY = [(148, 13312), (132, 16384), (148, 9088), (148, 6144)]
+GEOMETRY = [(148, 13312), (132, 16384), (148, 9088), (148, 8192)]
 PART_FLOATS = 1280  # per-CTA partial sums the kernel holds for one phase
 
 
@@ -134,6 +134,17 @@ def test_plan_rejects_bad_arguments(grid, stage, cap):
     buf = (K.kie_seg_range * 16)() if cap else None
     st = L.kie_plan(ctypes.byref(cfg), grid, stage, ctypes.byref(info), buf, cap or 0)
     assert st == -1 and L.kie_last_error(None)
+
+
+def test_plan_stage_holds_an_attention_sub_block():
+    """A ring stage also carries 32 K or V rows of one head: 8 KiB at head_dim
+    128, 4 KiB at 64. Smaller stages are rejected before anything could copy
+    past one."""
+    K.plan(S.TINY, 148, 4096)  # head_dim 64
+    with pytest.raises(K.KieError) as ei:
+        K.plan(S.DENSE_2B, 148, 6144)  # head_dim 128
+    assert ei.value.status == -1 and "attention sub-block" in str(ei.value)
+    K.plan(S.DENSE_2B, 148, 8192)
 
 
 def test_plan_rejects_shapes_like_create():

@@ -597,7 +597,10 @@ kie_status kie_create(const kie_config* cfg, int device, kie_ctx** out) {
   const int optin = (int)prop.sharedMemPerBlockOptin;
   const int ns = kernel_max_stages();
   int sb = std::min(kMaxStageBytes, ((optin - fixed) / ns) & ~1023);
-  if (sb < 4096) return bail(fail(c, KIE_ERR_INVALID_ARG, "shape needs too much shared memory"));
+  // a stage holds a weight tile (at least 4 KiB) or one attention sub-block
+  // of K or V rows (kAttnSub positions x head_dim fp16)
+  if (sb < std::max(4096, kAttnSub * dh * 2))
+    return bail(fail(c, KIE_ERR_INVALID_ARG, "shape needs too much shared memory"));
   c->n_stages = ns;
   c->stage_bytes = sb;
   c->smem = kernel_smem_bytes(vf, 4 * k.n_layers + 1, ns, sb);
@@ -610,7 +613,11 @@ kie_status kie_create(const kie_config* cfg, int device, kie_ctx** out) {
           cudaSuccess ||
       per_sm < 1)
     return bail(fail(c, KIE_ERR_CUDA, "kernel does not fit on an SM (smem %d)", c->smem));
-  c->grid = c->sms;  // one CTA per SM; the ring takes the SM's shared memory
+  // one CTA per SM (the ring takes the SM's shared memory), and no more CTAs
+  // than residual rows: every CTA publishes residual rows in every layer, and
+  // the flagged scratch words are reused layer after layer on the strength of
+  // that (a CTA cannot run a layer ahead of one that has not yet read them)
+  c->grid = std::min(c->sms, d);
   if ((d + c->grid - 1) / c->grid > kMaxOwnRows)
     return bail(fail(c, KIE_ERR_INVALID_ARG, "d_model %d over %d CTAs exceeds %d residual rows per CTA", d,
                      c->grid, kMaxOwnRows));
@@ -697,6 +704,9 @@ kie_status kie_plan(const kie_config* cfg, int32_t grid, int32_t stage_bytes, ki
   if (grid < 1) return fail(nullptr, KIE_ERR_INVALID_ARG, "grid %d < 1", grid);
   if (stage_bytes < 4096 || stage_bytes % 16)
     return fail(nullptr, KIE_ERR_INVALID_ARG, "stage_bytes %d: at least 4096 and a multiple of 16", stage_bytes);
+  if (cfg && stage_bytes < kAttnSub * cfg->head_dim * 2)
+    return fail(nullptr, KIE_ERR_INVALID_ARG, "stage_bytes %d: below one attention sub-block (%d B)", stage_bytes,
+                kAttnSub * cfg->head_dim * 2);
   Plan plan;
   if (kie_status ps = make_plan(nullptr, *cfg, grid, stage_bytes, plan)) return ps;
   const int per_cta = cfg->n_layers * plan.slots + 1;
@@ -1097,8 +1107,9 @@ kie_status launch_on(kie_ctx* c, const Run& r, unsigned char* sync_base, size_t 
   if (ctl.err) {
     c->poisoned = true;
     static const char* where[] = {"?", "grid barrier", "ring stage (full)", "ring stage (empty)",
-                                  "expert routing hand-off", "device check", "flagged input wait"};
-    const int w = (ctl.err_where >= 1 && ctl.err_where <= 6) ? ctl.err_where : 0;
+                                  "expert routing hand-off", "device check", "flagged input wait",
+                                  "ring tile larger than a stage"};
+    const int w = (ctl.err_where >= 1 && ctl.err_where <= 7) ? ctl.err_where : 0;
     return fail(c, (kie_status)ctl.err, "device %s at %s (cta %d, step %d); context poisoned",
                 ctl.err == KIE_ERR_TIMEOUT ? "timeout" : "check failed", where[w], ctl.err_cta,
                 ctl.err_step);

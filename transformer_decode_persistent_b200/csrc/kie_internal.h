@@ -73,7 +73,8 @@ struct Ctrl {
   int err_cta;           // CTA that recorded the error
   int err_step;          // decode step
   int err_where;         // 1 grid barrier, 2 ring full-wait, 3 ring empty-wait,
-                         // 4 route wait, 5 device check, 6 flagged-word wait
+                         // 4 route wait, 5 device check, 6 flagged-word wait,
+                         // 7 ring tile larger than a stage
   int final_token;       // pending token after the last step
   int pad;
 };

@@ -473,6 +473,11 @@ struct Producer {
 
   // Put tile tt (bytes at src; 0 bytes = an empty tile) into this lane's stage.
   __device__ bool put(unsigned tt, const void* src, unsigned bytes) {
+    if (bytes > (unsigned)P.stage_bytes) {  // never copy past the stage (the host sizes stages to fit)
+      record_error(P, kErrDevice, 7, step);
+      sc->abort = 1;
+      return false;
+    }
     const unsigned n = tt / P.n_stages;
     if (n > 0 && !wait_bar(P, sc, &sc->empty[lane], (n - 1) & 1u, 3, step)) return false;
     mbar_expect_tx(&sc->full[lane], bytes);  // with 0 bytes this arrival completes the phase
