@@ -224,7 +224,9 @@ def summarize_phase_trace(t: np.ndarray, n_layers: int) -> dict:
     barrier last in each step as arrival, release, release, release).
 
     Per CTA and step, each phase kind's input wait (start -> input ready),
-    tile time and epilogue time are summed over the layers; the figures are
+    tile time and epilogue time are summed over the layers (attention: the
+    wait for q and this token's k/v, the CTA's own units, the cross-CTA chunk
+    merge); the figures are
     medians over CTAs of the per-step mean. The step time is the interval
     between consecutive barrier releases (median over CTAs); the wait share is
     the phases' input waits plus the barrier wait over the step time."""

@@ -53,9 +53,10 @@ def test_static_scratch_decode_equals_decode_on_two_calls():
 
 
 def test_static_scratch_rejects_models_that_do_not_fit():
-    # 256 query heads of 128 dims over 64 KV heads need about 1 MB of scratch
-    s = S.Shape("wide-heads", n_layers=1, d_model=64, n_heads=256, n_kv_heads=64, head_dim=128,
-                ffn=64, vocab=100, max_ctx=1024)
+    # 32 query heads of 128 dims over 8 KV heads at up to 4480 positions keep
+    # 20 attention chunk records per head: about 0.75 MB of scratch
+    s = S.Shape("wide-heads", n_layers=1, d_model=256, n_heads=32, n_kv_heads=8, head_dim=128,
+                ffn=256, vocab=100, max_ctx=4480)
     e = Engine(s)
     e.load_weights(S.make_weights(s, seed=1, cache=False))
     import torch

@@ -49,6 +49,8 @@ struct kie_ctx {
   int xplane = 0;          // float offset of the input vector's second plane
   int vec_floats = 0;
   int gbuf_off = 0;
+  int rslice_off = 0;      // MoE router slice (floats into the vector buffer)
+  int rslice_rows = 0;
   int smem = 0;
   int max_chunks = 0;
   int hbuf = 0;
@@ -385,7 +387,7 @@ kie_status make_plan(kie_ctx* c, const kie_config& k, int G, int sb, Plan& plan)
 // The region cleared before every launch: control block, attention arrival
 // counters and the flagged scratch words (see Params).
 struct SyncLayout {
-  size_t fx, fq, fo, fh, fcand, apart, total;
+  size_t fx, fq, fo, fh, fcand, apart, froute, total;
 };
 
 SyncLayout sync_layout(const kie_config& k, int grid, int hbuf, int max_chunks) {
@@ -398,6 +400,7 @@ SyncLayout sync_layout(const kie_config& k, int grid, int hbuf, int max_chunks) 
   L.fh = off;    off += (size_t)hbuf * 8;
   L.fcand = off; off += (size_t)grid * 4 * 8;
   L.apart = off; off += (size_t)k.n_heads * max_chunks * (k.head_dim + 4) * 8;
+  L.froute = off; off += k.n_experts ? (size_t)(k.n_experts + 1) * ((grid + 1) & ~1) * 8 : 0;
   L.total = off;
   return L;
 }
@@ -410,6 +413,7 @@ void set_sync_params(Params& P, unsigned char* base, const SyncLayout& L) {
   P.fo = reinterpret_cast<unsigned long long*>(base + L.fo);
   P.fh = reinterpret_cast<unsigned long long*>(base + L.fh);
   P.fcand = reinterpret_cast<unsigned long long*>(base + L.fcand);
+  P.froute = reinterpret_cast<unsigned long long*>(base + L.froute);
 }
 
 // Shape checks shared by kie_create and kie_plan (messages via kie_last_error(NULL)).
@@ -590,6 +594,12 @@ kie_status kie_create(const kie_config* cfg, int device, kie_ctx** out) {
   vf = (vf + 3) & ~3;
   c->gbuf_off = vf;           // then d fp16 norm-gain values
   vf += ((d / 2) + 3) & ~3;
+  // MoE: then this layer's router columns of the CTA's residual rows, fp16
+  // [E][rslice_rows] (for the router partial sums of the output projection)
+  const int grid = std::min(c->sms, d);
+  c->rslice_off = vf;
+  c->rslice_rows = (d + grid - 1) / grid;
+  if (moe) vf += ((k.n_experts * c->rslice_rows + 1) / 2 + 3) & ~3;
   c->vec_floats = vf;
   // kRingStages ring stages (two per consumer warp) of the largest size that
   // fits, in 1 KiB steps, at most 16 KiB
@@ -617,7 +627,9 @@ kie_status kie_create(const kie_config* cfg, int device, kie_ctx** out) {
   // than residual rows: every CTA publishes residual rows in every layer, and
   // the flagged scratch words are reused layer after layer on the strength of
   // that (a CTA cannot run a layer ahead of one that has not yet read them)
-  c->grid = std::min(c->sms, d);
+  c->grid = grid;
+  if (moe && c->grid > kRouteMaxGrid)
+    return bail(fail(c, KIE_ERR_INVALID_ARG, "MoE routing supports at most %d CTAs", kRouteMaxGrid));
   if ((d + c->grid - 1) / c->grid > kMaxOwnRows)
     return bail(fail(c, KIE_ERR_INVALID_ARG, "d_model %d over %d CTAs exceeds %d residual rows per CTA", d,
                      c->grid, kMaxOwnRows));
@@ -1074,6 +1086,8 @@ Params make_params(const kie_ctx* c, const Run& r, unsigned char* sync_base) {
   P.n_stages = c->n_stages; P.stage_bytes = c->stage_bytes; P.vec_floats = c->vec_floats;
   P.xplane = c->xplane;
   P.gbuf_off = c->gbuf_off;
+  P.rslice_off = c->rslice_off;
+  P.rslice_rows = c->rslice_rows;
   P.samp_temp = r.temperature; P.samp_p = r.top_p; P.samp_k = r.top_k; P.samp_seed = r.seed;
   P.fsamp = c->fsamp;
   P.lm_logits = c->lm_logits;

@@ -23,6 +23,7 @@ constexpr int kMaxHeadsPerGroup = 4;                   // query heads per KV hea
 constexpr int kMaxTopK = 8;                            // routed experts per token
 constexpr int kAttnSub = 32;                           // positions per attention sub-block
 constexpr int kMaxExperts = 256;
+constexpr int kRouteMaxGrid = 192;                     // MoE: CTAs whose router partials one warp sums (3 pairs a lane)
 constexpr int kMaxOwnRows = 64;                        // residual rows a CTA keeps in shared memory
 constexpr int kSampleK = 64;                           // largest top-k of in-kernel sampling
 constexpr int kSampleMaxGrid = 160;                    // CTAs whose candidates one CTA can merge
@@ -116,6 +117,8 @@ struct Params {
   unsigned long long* fh;     // [hbuf] FFN hidden (dense: ff; MoE: ffs + top_k*ffe)
   unsigned long long* fcand;  // [grid][3] LM-head candidates: best value, its index, second value
   unsigned long long* apart;  // attention chunk records [hq][max_chunks][dh + 4]: (max, sum), pad, acc[dh]
+  unsigned long long* froute; // MoE: router partials [E + 1][grid]: row e < E = this CTA's residual rows'
+                              // share of router logit e (before the RMSNorm factor); row E = their sum of squares
   Ctrl* ctrl;
   int max_chunks;
   // run
@@ -142,6 +145,8 @@ struct Params {
   int stage_bytes;
   int vec_floats;   // shared vector buffer, including the norm-gain buffer at gbuf_off
   int gbuf_off;     // float offset of the fp16 norm-gain buffer inside the vector buffer
+  int rslice_off;   // MoE: float offset of the fp16 router slice [E][own rows] inside the vector buffer
+  int rslice_rows;  // MoE: own-row capacity of each expert's slice
   int xplane;       // float offset of the second-half plane of the input vector (see Consumer::xv)
 };
 

@@ -179,6 +179,11 @@ __device__ __forceinline__ void ld_flag2(const unsigned long long* p, unsigned l
                                          unsigned long long& b) {
   asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
 }
+__device__ __forceinline__ unsigned long long ld_flag1(const unsigned long long* p) {
+  unsigned long long a;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(a) : "l"(p) : "memory");
+  return a;
+}
 __device__ __forceinline__ unsigned fepoch(unsigned long long w) { return (unsigned)(w >> 32); }
 __device__ __forceinline__ float fval(unsigned long long w) { return __uint_as_float((unsigned)w); }
 // consumer-only barrier (named barrier 1 over the 224 consumer threads)
@@ -427,10 +432,18 @@ __device__ bool wait_bar(const Params& P, SmemCtl* sc, uint64_t* b, unsigned par
 // tiles of sub-range k land on the same consumer warp. The row of `pos` itself
 // is written during this step and is never in a tile; the warp that owns it
 // reads it directly.
+//
+// A unit is normally one KV head's chunk for all the query heads it serves
+// (its K/V rows are read once). When the query heads' units of every chunk
+// fit in one wave of CTAs (short context with grouped heads), each query head
+// becomes a unit of its own instead: the group's K/V rows are then read once
+// per query head, a small cost at short context, and the work of a group is
+// spread over as many CTAs as it has query heads. Per head the arithmetic and
+// its order are the same either way.
 struct AttnPlan {
-  int T, per, pw, nsb, nchk, units;
+  int T, per, pw, nsb, nchk, units, split;
 };
-__device__ __forceinline__ AttnPlan attn_plan(int pos, int hk, int grid) {
+__device__ __forceinline__ AttnPlan attn_plan(int pos, int hk, int hq, int grid) {
   constexpr int kUnitMin = kConsumerWarps * kAttnSub;
   AttnPlan a;
   a.T = pos + 1;
@@ -440,8 +453,30 @@ __device__ __forceinline__ AttnPlan attn_plan(int pos, int hk, int grid) {
   a.pw = per / kConsumerWarps;
   a.nsb = a.pw / kAttnSub;
   a.nchk = (a.T + per - 1) / per;
-  a.units = hk * a.nchk;
+  a.split = (hq > hk && hq * a.nchk <= grid) ? 1 : 0;
+  a.units = (a.split ? hq : hk) * a.nchk;
   return a;
+}
+// Unit u: KV head g, chunk ch, query heads h_lo .. h_lo + nh - 1. KV head g
+// serves query heads ceil(g hq / hk) .. ceil((g + 1) hq / hk) - 1, so query
+// head q belongs to KV head floor(q hk / hq).
+struct AttnUnit {
+  int g, ch, h_lo, nh;
+};
+__device__ __forceinline__ AttnUnit attn_unit(const AttnPlan& a, int u, int hk, int hq) {
+  AttnUnit r;
+  const int idx = u / a.nchk;
+  r.ch = u - idx * a.nchk;
+  if (a.split) {
+    r.h_lo = idx;
+    r.nh = 1;
+    r.g = (int)(((long long)idx * hk) / hq);
+  } else {
+    r.g = idx;
+    r.h_lo = (idx * hq + hk - 1) / hk;
+    r.nh = ((idx + 1) * hq + hk - 1) / hk - r.h_lo;
+  }
+  return r;
 }
 __device__ __forceinline__ int attn_units_of(const AttnPlan& a, int cta, int grid) {
   return a.units > cta ? (a.units - cta + grid - 1) / grid : 0;
@@ -473,11 +508,6 @@ struct Producer {
 
   // Put tile tt (bytes at src; 0 bytes = an empty tile) into this lane's stage.
   __device__ bool put(unsigned tt, const void* src, unsigned bytes) {
-    if (bytes > (unsigned)P.stage_bytes) {  // never copy past the stage (the host sizes stages to fit)
-      record_error(P, kErrDevice, 7, step);
-      sc->abort = 1;
-      return false;
-    }
     const unsigned n = tt / P.n_stages;
     if (n > 0 && !wait_bar(P, sc, &sc->empty[lane], (n - 1) & 1u, 3, step)) return false;
     mbar_expect_tx(&sc->full[lane], bytes);  // with 0 bytes this arrival completes the phase
@@ -506,7 +536,7 @@ struct Producer {
   // K/V rows of this CTA's attention units of layer l (see attn_plan).
   __device__ bool issue_attn(int l, int pos) {
     const int G = gridDim.x, ns = P.n_stages, hk = P.hk, dh = P.dh;
-    const AttnPlan ap = attn_plan(pos, hk, G);
+    const AttnPlan ap = attn_plan(pos, hk, P.hq, G);
     const int nu = attn_units_of(ap, blockIdx.x, G);
     const int per_unit = ap.nsb * kAttnTilesPerRound;
     const int ntiles = nu * per_unit;
@@ -520,7 +550,8 @@ struct Producer {
       const int k = ti % kConsumerWarps;
       const bool isv = ti >= kConsumerWarps;
       const int u = blockIdx.x + uo * G;
-      const int g = u / ap.nchk, ch = u - g * ap.nchk;
+      const AttnUnit au = attn_unit(ap, u, hk, P.hq);
+      const int g = au.g, ch = au.ch;
       const int j0 = ch * ap.per, j1 = min(ap.T, j0 + ap.per);
       const int wj0 = j0 + k * ap.pw, wj1 = min(j1, wj0 + ap.pw);
       const int jb = wj0 + b * kAttnSub;
@@ -549,7 +580,22 @@ struct Producer {
     return true;
   }
 
+  // Every tile is at most g x kc halves of its segment shape, or one attention
+  // sub-block of K or V rows; the host sizes the stages to hold both. Checked
+  // once here rather than per copy (the copy path is inlined at every issue
+  // site): a plan that breaks it copies nothing.
+  __device__ bool tiles_fit() const {
+    bool fit = kAttnSub * P.dh * 2 <= P.stage_bytes;
+    for (int k = 0; k < SK_COUNT; ++k) fit = fit && P.shp[k].g * P.shp[k].kc * 2 <= P.stage_bytes;
+    return fit;
+  }
+
   __device__ void run() {
+    if (!tiles_fit()) {
+      if (lane == 0) record_error(P, kErrDevice, 7, 0);
+      sc->abort = 1;
+      return;
+    }
     bool ok = true;
     unsigned route_round = 0;
     for (step = 0; ok && step < P.n_steps; ++step) {
@@ -704,7 +750,6 @@ struct Consumer {
       : P(p), sc(s), part(pa), vec(v), ring(r), tid(threadIdx.x), warp(threadIdx.x >> 5),
         lane(threadIdx.x & 31), dc(d) {}
 
-  __device__ __forceinline__ int ap_nchk(int pos) const { return attn_plan(pos, P.hk, gridDim.x).nchk; }
 
   // Phase trace (KIE_TRACE builds): per CTA and step, one record of four
   // %globaltimer stamps per phase -- phase start (before its input wait),
@@ -1162,14 +1207,17 @@ struct Consumer {
   // the ring (see attn_plan); each warp handles one sub-range of each of the
   // CTA's units, lanes over head dims for both q.k (butterfly transpose-reduce
   // of 32 positions) and the V sum. The warps' (max, sum, acc) partials are
-  // merged in shared memory; a head spanning several CTAs is finished by the
-  // last of them (arrival counter per KV head) from per-CTA partials.
+  // merged in shared memory; a head split into chunks over several CTAs is
+  // finished by the CTA of its chunk 0 from the flagged chunk records.
+  // Trace stamps of the phase (KIE_TRACE builds): input = q and this token's
+  // k/v of the first unit arrived, tiles = every unit's sub-ranges done and
+  // merged in the CTA, epilogue (by the caller) = cross-CTA chunk merges done.
   template <int DH>
-  __device__ void attention(int l, int pos) {
+  __device__ void attention(int l, int pos, int ph) {
     constexpr int DPL = DH / 32;   // head dims per lane
     constexpr int WS = DH + 4;     // partial record: m, l, pad, pad, acc[DH]
     const int hk = P.hk, hq = P.hq, G = gridDim.x;
-    const AttnPlan ap = attn_plan(pos, hk, G);
+    const AttnPlan ap = attn_plan(pos, hk, hq, G);
     const int nu = attn_units_of(ap, blockIdx.x, G);
     const int vs = (int)((warp + kConsumerWarps - (int)(tbase % kConsumerWarps)) % kConsumerWarps);
     float* qs = vec;                                              // [nh][DH]
@@ -1178,9 +1226,8 @@ struct Consumer {
     const uint32_t ring_s = su32(ring);
     for (int uo = 0; uo < nu; ++uo) {
       const int u = blockIdx.x + uo * G;
-      const int g = u / ap.nchk, ch = u - g * ap.nchk;
-      const int h_lo = (g * hq + hk - 1) / hk;
-      const int nh = (((g + 1) * hq + hk - 1) / hk) - h_lo;
+      const AttnUnit au = attn_unit(ap, u, hk, hq);
+      const int g = au.g, ch = au.ch, h_lo = au.h_lo, nh = au.nh;
       const int j0 = ch * ap.per, j1 = min(ap.T, j0 + ap.per);
       const int wj0 = j0 + vs * ap.pw, wj1 = min(j1, wj0 + ap.pw);
       // q of this group's heads and this token's own k/v row (not in the ring)
@@ -1204,6 +1251,7 @@ struct Consumer {
         }
       }
       if (cbar_any(sc->abort != 0)) return;
+      if (uo == 0) tstamp(ph, 1);
       switch (nh) {
         case 1: attn_warp<DH, 1>(ap, uo, vs, wj0, wj1, pos, kpos, vpos, qs, wp, sbuf); break;
         case 2: attn_warp<DH, 2>(ap, uo, vs, wj0, wj1, pos, kpos, vpos, qs, wp, sbuf); break;
@@ -1244,17 +1292,17 @@ struct Consumer {
       }
       cbar();  // qs / wp are reused by the next unit
     }
+    if (nu == 0) tstamp(ph, 1);
+    tstamp(ph, 2);
     // A KV head split into chunks is finished by the CTA of its chunk 0. That
     // CTA merges only after it has published the records of all its own units,
     // so no CTA waits for a record that one of its later units would produce.
     if (ap.nchk > 1) {
       for (int uo = 0; uo < nu; ++uo) {
         const int u = blockIdx.x + uo * G;
-        const int g = u / ap.nchk, ch = u - g * ap.nchk;
-        if (ch != 0) continue;
-        const int h_lo = (g * hq + hk - 1) / hk;
-        const int nh = (((g + 1) * hq + hk - 1) / hk) - h_lo;
-        if (warp < nh) merge_chunks<DH>(h_lo + warp, ap.nchk, epoch(l));
+        const AttnUnit au = attn_unit(ap, u, hk, hq);
+        if (au.ch != 0) continue;
+        if (warp < au.nh) merge_chunks<DH>(au.h_lo + warp, ap.nchk, epoch(l));
       }
     }
     tbase += (unsigned)(nu * ap.nsb * kAttnTilesPerRound);
@@ -1334,9 +1382,9 @@ struct Consumer {
     for (int e = 0; e < DPL; e += 2) st_flag2(ob + e, acc[e] * inv, acc[e + 1] * inv, ep);
   }
 
-  __device__ void attention_dispatch(int l, int pos) {
-    if (P.dh == 128) attention<128>(l, pos);
-    else attention<64>(l, pos);
+  __device__ void attention_dispatch(int l, int pos, int ph) {
+    if (P.dh == 128) attention<128>(l, pos, ph);
+    else attention<64>(l, pos, ph);
   }
 
   // Copy the RoPE coefficients of this CTA's first kRopeStage q/k row pairs at
@@ -1409,6 +1457,44 @@ struct Consumer {
       sc->xown[r] = v;
       st_flag(fx + row, v, ep);
     }
+    if (which == 0 && P.E) router_partials(sd, ep);
+  }
+
+  // MoE router logit e = (R_e . (g * x)) / rms(x), with x the residual stream
+  // after the output projection and g the FFN RMSNorm gain. Both the dot
+  // product and the sum of squares split over the residual rows, so every CTA
+  // publishes its rows' share of each (flagged, row e of froute for logit e,
+  // row E for the squares) and the router needs no GEMV of its own: the
+  // FFN-up phase sums the grid's shares (route). The router columns of the
+  // rows were staged in shared memory by prefetch_router, and the gain by
+  // prefetch_gain.
+  __device__ void router_partials(const SegDesc& sd, unsigned ep) {
+    asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's gain copies
+    cbar();  // every row's x, every thread's gain copies and the staged router columns
+    const __half* rs = reinterpret_cast<const __half*>(vec + P.rslice_off);
+    const __half* gb = reinterpret_cast<const __half*>(vec + P.gbuf_off);
+    const int n = sd.nrows, cap = P.rslice_rows;
+    for (int e = warp; e <= P.E; e += kConsumerWarps) {
+      float a = 0.f;
+      for (int r = lane; r < n; r += 32) {
+        const float x = sc->xown[r];
+        a = e < P.E ? fmaf(__half2float(rs[e * cap + r]) * __half2float(gb[sd.row0 + r]), x, a) : fmaf(x, x, a);
+      }
+      a = warp_sum(a);
+      if (lane == 0) st_flag(P.froute + (size_t)e * ((gridDim.x + 1) & ~1u) + blockIdx.x, a, ep);
+    }
+  }
+
+  // Stage layer l's router columns of this CTA's residual rows in shared
+  // memory ([E][rslice_rows] fp16), during the output projection's input wait.
+  __device__ void prefetch_router(int l, const SegDesc& sd) {
+    __half* rs = reinterpret_cast<__half*>(vec + P.rslice_off);
+    const __half* R = P.router + (size_t)l * P.E * P.d + sd.row0;
+    const int n = sd.nrows, cap = P.rslice_rows;
+    for (int i = tid; i < P.E * n; i += kConsumerThreads) {
+      const int e = i / n, r = i - e * n;
+      rs[e * cap + r] = R[(size_t)e * P.d + r];
+    }
   }
 
   // SwiGLU epilogue over interleaved (gate, up) rows: h[hoff + row0/2 + j] = w * silu(g) * u
@@ -1427,19 +1513,75 @@ struct Consumer {
     }
   }
 
-  // MoE router, computed redundantly by every CTA from the normalised input in vec.
+  // MoE routing, decided identically by every CTA: the logits are the sums of
+  // the grid's flagged router partials (router_partials), added in one fixed
+  // order (warp e % 7 sums row e, each lane its CTAs 2 lane + 64 k, k < 3,
+  // then a butterfly), so every CTA takes the same decision from the same
+  // words. Rows are polled kRouteRows at a time, all loads issued first.
+  static constexpr int kRouteRows = 4;
   __device__ void route(int l) {
-    const __half* R = P.router + (size_t)l * P.E * P.d;
-    for (int e = warp; e < P.E; e += kConsumerWarps) {
-      const __half* row = R + (size_t)e * P.d;
-      float a = 0.f;
-      for (int c = lane; c < P.d / 8; c += 32) {
-        const uint4 wv = *reinterpret_cast<const uint4*>(row + c * 8);
-        a = dot8(wv, *reinterpret_cast<const float4*>(xv(c * 8)),
-                 *reinterpret_cast<const float4*>(xv(c * 8 + 4)), a);
+    const int G = gridDim.x, E = P.E, gp = (G + 1) & ~1;  // rows padded to pairs
+    const unsigned ep = epoch(l);
+    // warp-uniform trip count: the polls' votes need every lane
+    for (int e0 = warp; e0 <= E; e0 += kConsumerWarps * kRouteRows) {
+      unsigned long long w[kRouteRows][3][2];
+#pragma unroll
+      for (int b = 0; b < kRouteRows; ++b) {
+        const int e = e0 + b * kConsumerWarps;
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+          const int c = 2 * lane + 64 * k;
+          w[b][k][0] = w[b][k][1] = fpack(0.f, ep);
+          if (e <= E && c < G) {
+            const unsigned long long* src = P.froute + (size_t)e * gp + c;
+            if (c + 1 < G) ld_flag2(src, w[b][k][0], w[b][k][1]);
+            else w[b][k][0] = ld_flag1(src);
+          }
+        }
       }
-      a = warp_sum(a);
-      if (lane == 0) part[e] = a * norm_scale();
+      unsigned long long t0 = 0;
+      for (unsigned it = 0;; ++it) {
+        bool stale = false;
+#pragma unroll
+        for (int b = 0; b < kRouteRows; ++b) {
+          const int e = e0 + b * kConsumerWarps;
+#pragma unroll
+          for (int k = 0; k < 3; ++k) {
+            const int c = 2 * lane + 64 * k;
+            if (fepoch(w[b][k][0]) != ep || fepoch(w[b][k][1]) != ep) {
+              stale = true;
+              const unsigned long long* src = P.froute + (size_t)e * gp + c;
+              if (c + 1 < G) ld_flag2(src, w[b][k][0], w[b][k][1]);
+              else w[b][k][0] = ld_flag1(src);
+            }
+          }
+        }
+        if (!__any_sync(0xffffffffu, stale)) break;
+        if (it == 0) {
+          t0 = gtimer();
+        } else if ((it & 31) == 0) {
+          bool give_up = false;
+          if (sc->abort || ld_relaxed(&P.ctrl->abort)) {
+            give_up = true;
+          } else if (gtimer() - t0 > P.timeout_ns) {
+            record_error(P, kErrTimeout, 4, step);
+            give_up = true;
+          }
+          if (__any_sync(0xffffffffu, give_up)) {
+            sc->abort = 1;
+            break;
+          }
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < kRouteRows; ++b) {
+        float a = 0.f;
+#pragma unroll
+        for (int k = 0; k < 3; ++k) a += fval(w[b][k][0]) + fval(w[b][k][1]);
+        a = warp_sum(a);
+        const int e = e0 + b * kConsumerWarps;
+        if (lane == 0 && e <= E) part[e < E ? e : 2 * kMaxExperts] = a;
+      }
     }
     cbar();
     if (warp == 0) {
@@ -1447,6 +1589,9 @@ struct Consumer {
       // denominator cancels in the renormalisation), larger first and the
       // lower expert index on ties; a chosen expert is struck out with -1
       float* pr = part + kMaxExperts;
+      const float inv = 1.0f / sqrtf(part[2 * kMaxExperts] / (float)P.d + P.eps);
+      for (int e = lane; e < P.E; e += 32) part[e] *= inv;
+      __syncwarp();
       float mx = -INFINITY;
       for (int e = lane; e < P.E; e += 32) mx = fmaxf(mx, part[e]);
       mx = warp_max(mx);
@@ -1470,6 +1615,10 @@ struct Consumer {
             bv = ov;
             bi = oi;
           }
+        }
+        if (bi >= P.E) {  // no orderable candidate (a non-finite logit): stop, with a valid index
+          bi = k;
+          if (lane == 0) record_error(P, kErrDevice, 5, step);
         }
         if (lane == 0) {
           re[k] = bi;
@@ -1528,13 +1677,13 @@ struct Consumer {
             prefetch_gain(P.mlp_norm + (size_t)l * P.d);
             break;
           case PH_O:
+            if (P.E) prefetch_router(l, dc.at(l, 1));
             load_vec(P.fo, epoch(l), P.hq * P.dh);
             break;
           case PH_UP:
-            load_norm(P.fx, epoch(l), nullptr, P.d);
-            if (l + 1 < P.L) prefetch_gain(P.attn_norm + (size_t)(l + 1) * P.d);
-            else prefetch_gain(lm ? P.final_norm : P.attn_norm);
             if (P.E) {
+              // routing first: the producer issues the routed experts' tiles
+              // while this CTA loads x and runs the shared expert
               const int* pick = sc->route_e[route_round % kRouteRing];
               route(l);
               for (int k = 0; k < P.top_k; ++k) {
@@ -1542,6 +1691,9 @@ struct Consumer {
                 rw[k] = sc->route_w[k];
               }
             }
+            load_norm(P.fx, epoch(l), nullptr, P.d);
+            if (l + 1 < P.L) prefetch_gain(P.attn_norm + (size_t)(l + 1) * P.d);
+            else prefetch_gain(lm ? P.final_norm : P.attn_norm);
             break;
           case PH_DOWN:
             load_vec(P.fh, epoch(l), P.E ? P.ffs + P.top_k * P.ffe : P.ff);
@@ -1553,43 +1705,42 @@ struct Consumer {
           default:
             break;
         }
-        tstamp(ph, 1);
+        if (kind != PH_ATTN) tstamp(ph, 1);  // attention stamps its own input and tile times
         // ---- 2. tiles
         if (kind == PH_ATTN) {
-          attention_dispatch(l, pos);
-        } else if (kind == PH_LM || (kind == PH_UP && !P.E)) {
-          // the LM head and the dense gate/up run in row chunks that fit the
-          // partial-sum buffer, each chunk followed by its epilogue (the
-          // chunks are whole tile groups: contiguous in the tape and in the
-          // producer's tile order)
-          const SegDesc& full = kind == PH_LM ? dc.at(P.L, 0) : dc.at(l, 2);
-          const SegShape& sh = P.shp[kind == PH_LM ? SK_LM : SK_GU];
-          const int crows = max(sh.g, (kPartFloats / sh.nk) / sh.g * sh.g);
-          const float inv = norm_scale();
+          attention_dispatch(l, pos, ph);
+        } else {
+          // The LM head and the dense gate/up run in row chunks that fit the
+          // partial-sum buffer, each chunk followed by its epilogue (the chunks
+          // are whole tile groups: contiguous in the tape and in the
+          // producer's tile order). MoE phases run the shared expert and the
+          // routed experts as segments. All go through this one run_segment
+          // call site.
+          const bool chunked = kind == PH_LM || (kind == PH_UP && !P.E);
+          const SegDesc& cfull = kind == PH_LM ? dc.at(P.L, 0) : dc.at(l, 2);
+          const int csk = kind == PH_LM ? SK_LM : SK_GU;
+          const SegShape& csh = P.shp[csk];
+          const int crows = chunked ? max(csh.g, (kPartFloats / csh.nk) / csh.g * csh.g) : 1;
+          const int nseg = chunked ? (cfull.nrows + crows - 1) / crows
+                                   : ((P.E && (kind == PH_UP || kind == PH_DOWN)) ? 1 + P.top_k : 1);
+          const float inv = chunked ? norm_scale() : 0.f;
           float v1 = -INFINITY, v2 = -INFINITY;
           int i1 = INT_MAX;
-          for (int r0 = 0; r0 < full.nrows; r0 += crows) {
-            const SegDesc sub{full.off + (unsigned long long)r0 * sh.K * 2, full.row0 + r0,
-                              min(crows, full.nrows - r0)};
-            run_segment(sub, sh, vec, 0, sh.nk, 0);
-            cbar();
-            if (kind == PH_LM) epi_lm_rows(sub, r0, inv, v1, i1, v2);
-            else epi_swiglu(sub, 0, sh.nk, 0, 1.0f, epoch(l));
-            cbar();  // the partial sums are reused by the next chunk
-          }
-          if (kind == PH_LM) lm_candidates(full, v1, i1, v2);
-        } else {
-          const int nseg = (P.E && (kind == PH_UP || kind == PH_DOWN)) ? 1 + P.top_k : 1;
           int pnext = 0;
           for (int si = 0; si < nseg; ++si) {
+            SegDesc sub;
             const SegDesc* sd;
             int sk, voff = 0, pbase = 0, pstride, kjbase = 0;
-            if (kind == PH_QKV) { sd = &dc.at(l, 0); sk = SK_QKV; }
+            if (chunked) {
+              const int r0 = si * crows;
+              sub = SegDesc{cfull.off + (unsigned long long)r0 * csh.K * 2, cfull.row0 + r0,
+                            min(crows, cfull.nrows - r0)};
+              sd = &sub;
+              sk = csk;
+            } else if (kind == PH_QKV) { sd = &dc.at(l, 0); sk = SK_QKV; }
             else if (kind == PH_O) { sd = &dc.at(l, 1); sk = SK_O; }
-            else if (kind == PH_LM) { sd = &dc.at(P.L, 0); sk = SK_LM; }
             else if (kind == PH_UP) {
-              if (!P.E) { sd = &dc.at(l, 2); sk = SK_GU; }
-              else if (si == 0) { sd = &dc.at(l, 2); sk = SK_SGU; }
+              if (si == 0) { sd = &dc.at(l, 2); sk = SK_SGU; }
               else { sd = &dc.at(l, 4 + re[si - 1]); sk = SK_EGU; pbase = pnext; rpb[si - 1] = pnext; }
             } else {  // PH_DOWN
               if (!P.E) { sd = &dc.at(l, 3); sk = SK_DOWN; }
@@ -1605,11 +1756,17 @@ struct Consumer {
                                                : P.shp[sk].nk;
             run_segment(*sd, P.shp[sk], vec + voff / 2, pbase, pstride, kjbase);
             pnext = pbase + sd->nrows * P.shp[sk].nk;
-            if (kind == PH_UP && P.E && si == 0) pnext = sd->nrows * P.shp[sk].nk;
+            if (chunked) {
+              cbar();
+              if (kind == PH_LM) epi_lm_rows(sub, si * crows, inv, v1, i1, v2);
+              else epi_swiglu(sub, 0, csh.nk, 0, 1.0f, epoch(l));
+              cbar();  // the partial sums are reused by the next chunk
+            }
           }
+          if (kind == PH_LM) lm_candidates(cfull, v1, i1, v2);
         }
         cbar();
-        tstamp(ph, 2);
+        if (kind != PH_ATTN) tstamp(ph, 2);
         // ---- 3. epilogue
         switch (kind) {
           case PH_QKV:
