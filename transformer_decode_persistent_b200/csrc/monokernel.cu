@@ -813,8 +813,9 @@ struct Consumer {
   // All of the batch's loads are issued before any epoch is checked, and the
   // groups still stale are re-polled together, so a thread waits about one L2
   // round trip per batch instead of one per group. Bounded: on abort or
-  // deadline it flags the CTA and leaves zeros.
-  static constexpr int kLoadBatch = 8;
+  // deadline it flags the CTA and leaves zeros. Four groups a thread (a
+  // 3584-float vector in one batch) measured fastest among 2, 3, 4, 6 and 8.
+  static constexpr int kLoadBatch = 4;
   __device__ __forceinline__ void fetch_batch(const unsigned long long* src, unsigned ep, int n, int base,
                                               float4 (&v)[kLoadBatch]) {
     unsigned long long w[kLoadBatch][4];
