@@ -58,7 +58,7 @@ def _kernel_hash() -> str:
     """Hash of the decode kernel's code (comments and whitespace removed), so
     DRAM counters stay attached to the code they were taken on."""
     h = hashlib.sha256()
-    for f in ("monokernel.cu", "kie_internal.h"):
+    for f in ("monokernel.cuh", "kie_internal.h"):
         with open(os.path.join(ROOT, "transformer_decode_persistent_b200", "csrc", f)) as fh:
             src = fh.read()
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)

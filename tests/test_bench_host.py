@@ -19,7 +19,7 @@ def bench_in(tmp_path, monkeypatch):
     sys.path.insert(0, ROOT)
     import bench
     os.makedirs(tmp_path / CSRC)
-    for f in ("monokernel.cu", "kie_internal.h"):
+    for f in ("monokernel.cuh", "kie_internal.h"):
         shutil.copy(os.path.join(ROOT, CSRC, f), tmp_path / CSRC / f)
     os.makedirs(tmp_path / "profiles")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
@@ -29,7 +29,7 @@ def bench_in(tmp_path, monkeypatch):
 def test_kernel_hash_ignores_comments_and_whitespace(bench_in):
     bench, root = bench_in
     h0 = bench._kernel_hash()
-    p = root / CSRC / "monokernel.cu"
+    p = root / CSRC / "monokernel.cuh"
     src = p.read_text()
     p.write_text("// a new comment line\n/* and a\n block */\n" + src.replace("\n", "\n\n"))
     assert bench._kernel_hash() == h0

@@ -28,7 +28,15 @@
 namespace kie {
 int kernel_smem_bytes(int vec_floats, int n_desc, int n_stages, int stage_bytes);
 int kernel_max_stages();
-const void* kernel_entry();
+const void* kernel_entry_128_0();
+const void* kernel_entry_128_1();
+const void* kernel_entry_64_0();
+const void* kernel_entry_64_1();
+// the decode kernel compiled for this head_dim and FFN kind (decode_inst.cu)
+inline const void* kernel_entry(int head_dim, bool moe) {
+  if (head_dim == 128) return moe ? kernel_entry_128_1() : kernel_entry_128_0();
+  return moe ? kernel_entry_64_1() : kernel_entry_64_0();
+}
 }  // namespace kie
 
 using namespace kie;
@@ -614,12 +622,12 @@ kie_status kie_create(const kie_config* cfg, int device, kie_ctx** out) {
   c->n_stages = ns;
   c->stage_bytes = sb;
   c->smem = kernel_smem_bytes(vf, 4 * k.n_layers + 1, ns, sb);
-  if (cudaFuncSetAttribute(kernel_entry(), cudaFuncAttributeMaxDynamicSharedMemorySize, c->smem) !=
+  if (cudaFuncSetAttribute(kernel_entry(dh, moe), cudaFuncAttributeMaxDynamicSharedMemorySize, c->smem) !=
       cudaSuccess)
     return bail(fail(c, KIE_ERR_CUDA, "cudaFuncSetAttribute(smem=%d) failed: %s", c->smem,
                      cudaGetErrorString(cudaGetLastError())));
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel_entry(), kThreads, c->smem) !=
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel_entry(dh, moe), kThreads, c->smem) !=
           cudaSuccess ||
       per_sm < 1)
     return bail(fail(c, KIE_ERR_CUDA, "kernel does not fit on an SM (smem %d)", c->smem));
@@ -1104,7 +1112,7 @@ kie_status launch_on(kie_ctx* c, const Run& r, unsigned char* sync_base, size_t 
   CUDA_TRY(c, cudaMemsetAsync(sync_base, 0, sync_bytes, st));
   if (r.temperature > 0.f) CUDA_TRY(c, cudaMemsetAsync(c->fsamp, 0, c->fsamp_bytes, st));
   void* args[] = {&P};
-  cudaError_t e = cudaLaunchCooperativeKernel(kernel_entry(), dim3(c->grid), dim3(kThreads), args,
+  cudaError_t e = cudaLaunchCooperativeKernel(kernel_entry(c->cfg.head_dim, c->cfg.n_experts > 0), dim3(c->grid), dim3(kThreads), args,
                                               (size_t)c->smem, st);
   if (e != cudaSuccess) {
     cudaGetLastError();

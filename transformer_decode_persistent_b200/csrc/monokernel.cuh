@@ -388,7 +388,7 @@ __device__ __forceinline__ int key_index(unsigned long long k) { return (int)(0x
 
 // ---------------------------------------------------------------- errors
 
-__device__ void record_error(const Params& P, int code, int where, int step) {
+static __device__ void record_error(const Params& P, int code, int where, int step) {
   if (atomicCAS(&P.ctrl->err, 0, code) == 0) {
     P.ctrl->err_cta = blockIdx.x;
     P.ctrl->err_step = step;
@@ -402,7 +402,7 @@ __device__ void record_error(const Params& P, int code, int where, int step) {
 // `spin` waits with non-suspending probes: the producer's issuer lanes share
 // one warp and wait on different stages, and a lane suspended in try_wait
 // would hold up the others.
-__device__ bool wait_bar(const Params& P, SmemCtl* sc, uint64_t* b, unsigned parity, int where,
+static __device__ bool wait_bar(const Params& P, SmemCtl* sc, uint64_t* b, unsigned parity, int where,
                          int step, bool spin = false) {
   if (spin ? mbar_probe(b, parity) : mbar_test(b, parity)) return true;
   const unsigned long long t0 = gtimer();
@@ -485,6 +485,7 @@ constexpr int kAttnTilesPerRound = 2 * kConsumerWarps;
 
 // ---------------------------------------------------------------- producer
 
+template <bool MOE>
 struct Producer {
   // Each of the producer warp's lanes 0..n_stages-1 owns one ring stage and
   // issues the bulk copies of the tiles that land in it (tile t -> stage
@@ -602,7 +603,7 @@ struct Producer {
       for (int l = 0; ok && l < P.L; ++l) {
         ok = issue(dc.at(l, 0), P.shp[SK_QKV]) && issue_attn(l, P.pos0 + step) && issue(dc.at(l, 1), P.shp[SK_O]);
         if (!ok) break;
-        if (P.E == 0) {
+        if constexpr (!MOE) {
           ok = issue(dc.at(l, 2), P.shp[SK_GU]) && issue(dc.at(l, 3), P.shp[SK_DOWN]);
         } else {
           ok = issue(dc.at(l, 2), P.shp[SK_SGU]);
@@ -732,6 +733,9 @@ __device__ __forceinline__ float qk_partial(const float* q, uint2 r) {
   return t;
 }
 
+// HD: head_dim (64 or 128); MOE: routed-expert FFN. One kernel is compiled
+// per combination, so each model runs only its own code.
+template <int HD, bool MOE>
 struct Consumer {
   const Params& P;
   SmemCtl* sc;
@@ -1383,10 +1387,7 @@ struct Consumer {
     for (int e = 0; e < DPL; e += 2) st_flag2(ob + e, acc[e] * inv, acc[e + 1] * inv, ep);
   }
 
-  __device__ void attention_dispatch(int l, int pos, int ph) {
-    if (P.dh == 128) attention<128>(l, pos, ph);
-    else attention<64>(l, pos, ph);
-  }
+  __device__ void attention_dispatch(int l, int pos, int ph) { attention<HD>(l, pos, ph); }
 
   // Copy the RoPE coefficients of this CTA's first kRopeStage q/k row pairs at
   // position pos into shared memory (cp.async; load_norm's wait covers it).
@@ -1458,7 +1459,9 @@ struct Consumer {
       sc->xown[r] = v;
       st_flag(fx + row, v, ep);
     }
-    if (which == 0 && P.E) router_partials(sd, ep);
+    if constexpr (MOE) {
+      if (which == 0) router_partials(sd, ep);
+    }
   }
 
   // MoE router logit e = (R_e . (g * x)) / rms(x), with x the residual stream
@@ -1678,11 +1681,11 @@ struct Consumer {
             prefetch_gain(P.mlp_norm + (size_t)l * P.d);
             break;
           case PH_O:
-            if (P.E) prefetch_router(l, dc.at(l, 1));
+            if constexpr (MOE) prefetch_router(l, dc.at(l, 1));
             load_vec(P.fo, epoch(l), P.hq * P.dh);
             break;
           case PH_UP:
-            if (P.E) {
+            if constexpr (MOE) {
               // routing first: the producer issues the routed experts' tiles
               // while this CTA loads x and runs the shared expert
               const int* pick = sc->route_e[route_round % kRouteRing];
@@ -1697,7 +1700,7 @@ struct Consumer {
             else prefetch_gain(lm ? P.final_norm : P.attn_norm);
             break;
           case PH_DOWN:
-            load_vec(P.fh, epoch(l), P.E ? P.ffs + P.top_k * P.ffe : P.ff);
+            load_vec(P.fh, epoch(l), MOE ? P.ffs + P.top_k * P.ffe : P.ff);
             break;
           case PH_LM:
             load_norm(P.fx + P.d, epoch(P.L - 1), nullptr, P.d);
@@ -1717,13 +1720,13 @@ struct Consumer {
           // producer's tile order). MoE phases run the shared expert and the
           // routed experts as segments. All go through this one run_segment
           // call site.
-          const bool chunked = kind == PH_LM || (kind == PH_UP && !P.E);
+          const bool chunked = kind == PH_LM || (kind == PH_UP && !MOE);
           const SegDesc& cfull = kind == PH_LM ? dc.at(P.L, 0) : dc.at(l, 2);
           const int csk = kind == PH_LM ? SK_LM : SK_GU;
           const SegShape& csh = P.shp[csk];
           const int crows = chunked ? max(csh.g, (kPartFloats / csh.nk) / csh.g * csh.g) : 1;
           const int nseg = chunked ? (cfull.nrows + crows - 1) / crows
-                                   : ((P.E && (kind == PH_UP || kind == PH_DOWN)) ? 1 + P.top_k : 1);
+                                   : ((MOE && (kind == PH_UP || kind == PH_DOWN)) ? 1 + P.top_k : 1);
           const float inv = chunked ? norm_scale() : 0.f;
           float v1 = -INFINITY, v2 = -INFINITY;
           int i1 = INT_MAX;
@@ -1744,7 +1747,7 @@ struct Consumer {
               if (si == 0) { sd = &dc.at(l, 2); sk = SK_SGU; }
               else { sd = &dc.at(l, 4 + re[si - 1]); sk = SK_EGU; pbase = pnext; rpb[si - 1] = pnext; }
             } else {  // PH_DOWN
-              if (!P.E) { sd = &dc.at(l, 3); sk = SK_DOWN; }
+              if (!MOE) { sd = &dc.at(l, 3); sk = SK_DOWN; }
               else if (si == 0) { sd = &dc.at(l, 3); sk = SK_SDOWN; }
               else {
                 sd = &dc.at(l, 4 + P.E + re[si - 1]);
@@ -1753,7 +1756,7 @@ struct Consumer {
                 kjbase = P.shp[SK_SDOWN].nk + (si - 1) * P.shp[SK_EDOWN].nk;
               }
             }
-            pstride = (kind == PH_DOWN && P.E) ? P.shp[SK_SDOWN].nk + P.top_k * P.shp[SK_EDOWN].nk
+            pstride = (kind == PH_DOWN && MOE) ? P.shp[SK_SDOWN].nk + P.top_k * P.shp[SK_EDOWN].nk
                                                : P.shp[sk].nk;
             run_segment(*sd, P.shp[sk], vec + voff / 2, pbase, pstride, kjbase);
             pnext = pbase + sd->nrows * P.shp[sk].nk;
@@ -1777,14 +1780,14 @@ struct Consumer {
             epi_residual(dc.at(l, 1), P.shp[SK_O].nk, l == 0 ? erow : nullptr, 0, epoch(l));
             break;
           case PH_UP:
-            if (P.E) {
+            if constexpr (MOE) {
               epi_swiglu(dc.at(l, 2), 0, P.shp[SK_SGU].nk, 0, 1.0f, epoch(l));
               for (int k = 0; k < P.top_k; ++k)
                 epi_swiglu(dc.at(l, 4 + re[k]), rpb[k], P.shp[SK_EGU].nk, P.ffs + k * P.ffe, rw[k], epoch(l));
             }
             break;
           case PH_DOWN:
-            epi_residual(dc.at(l, 3), P.E ? P.shp[SK_SDOWN].nk + P.top_k * P.shp[SK_EDOWN].nk : P.shp[SK_DOWN].nk,
+            epi_residual(dc.at(l, 3), MOE ? P.shp[SK_SDOWN].nk + P.top_k * P.shp[SK_EDOWN].nk : P.shp[SK_DOWN].nk,
                          nullptr, 1, epoch(l));
             break;
           case PH_LM:  // run with the tiles, chunk by chunk
@@ -2047,6 +2050,7 @@ struct Consumer {
   }
 };
 
+template <int HD, bool MOE>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ Params P) {
   extern __shared__ __align__(1024) unsigned char smem[];
   SmemCtl* sc = reinterpret_cast<SmemCtl*>(smem);
@@ -2071,20 +2075,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   if (threadIdx.x >= kConsumerThreads) {
     const int lane = threadIdx.x - kConsumerThreads;
     if (lane < P.n_stages) {
-      Producer pr(P, sc, ring, lane, dc);
+      Producer<MOE> pr(P, sc, ring, lane, dc);
       pr.run();
     }
   } else {
-    Consumer cs(P, sc, part, vec, ring, dc);
+    Consumer<HD, MOE> cs(P, sc, part, vec, ring, dc);
     cs.run();
   }
 }
-
-// ---- host-side accessors used by the launcher
-int kernel_smem_bytes(int vec_floats, int n_desc, int n_stages, int stage_bytes) {
-  return smem_total(vec_floats, n_desc, n_stages, stage_bytes);
-}
-int kernel_max_stages() { return kMaxStages; }
-const void* kernel_entry() { return reinterpret_cast<const void*>(&decode_kernel); }
 
 }  // namespace kie
