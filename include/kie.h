@@ -54,7 +54,10 @@ typedef enum {
 } kie_status;
 
 /* Model shape. Dense models set n_experts = top_k = ffn_expert = ffn_shared = 0
- * and ffn > 0; MoE models set ffn = 0 and the four expert fields.
+ * and ffn > 0; MoE models set ffn = 0 and the expert fields; ffn_shared = 0 is
+ * a MoE layer without a shared expert (its shared.* tensors are then not
+ * passed to kie_load_weights). Each expert's rows are split over all CTAs, so
+ * every routing decision loads every SM with the same bytes.
  * Constraints: d_model, n_heads*head_dim, ffn, ffn_expert, ffn_shared multiples
  * of 8; head_dim 64 or 128; each KV head serves 1 to 4 query heads (query
  * head h reads KV head floor(h * n_kv_heads / n_heads)); max_ctx >= 1.
@@ -69,7 +72,7 @@ typedef enum {
  * head_dim and the FFN width; MoE: ffn_shared + top_k * ffn_expert) is held in
  * shared memory as fp32 beside the weight ring: about 40,000 values at most
  * (kie_create: "shape needs too much shared memory"). MoE: up to 256
- * experts, top_k up to 8. kie_load_weights and
+ * experts, top_k up to 8, at most 192 CTAs. kie_load_weights and
  * kie_plan reject a shape past these bounds with KIE_ERR_INVALID_ARG ("a CTA
  * would hold N partial sums (max 1280)"). */
 typedef struct {

@@ -170,16 +170,17 @@ def moe_ffn(xn, router, experts, shared, top_k: int) -> np.ndarray:
     """Routed SwiGLU experts plus an always-on shared expert, for one token.
 
     router: [E, d]; experts: list of (w_gate, w_up, w_down); shared: the same
-    triple. r = softmax(router . xn) over all E; the top-k experts (lowest
-    index on ties) are weighted by r_e / sum of the chosen r; the shared expert
-    is added with weight 1. Active-parameter streaming is what the pages say
+    triple, or None for a model without one (Qwen-class layers). r =
+    softmax(router . xn) over all E; the top-k experts (lowest index on ties)
+    are weighted by r_e / sum of the chosen r; the shared expert is added with
+    weight 1. Active-parameter streaming is what the pages say
     bounds MoE decode ("スケーリングをFrontier MoEモデルへ").
     """
     xn = f64(xn)
     r = softmax(xn @ f64(router).T)
     chosen = topk_lowest(r, top_k)
     wsum = sum(r[e] for e in chosen)
-    y = swiglu_ffn(xn, *shared)
+    y = swiglu_ffn(xn, *shared) if shared is not None else np.zeros_like(xn)
     for e in chosen:
         y = y + (r[e] / wsum) * swiglu_ffn(xn, *experts[e])
     return y
@@ -229,7 +230,7 @@ class Decoder:
                     self.W(p + f"experts.{e}.w_up"),
                     self.W(p + f"experts.{e}.w_down")) for e in range(s.n_experts)]
         shared = (self.W(p + "shared.w_gate"), self.W(p + "shared.w_up"),
-                  self.W(p + "shared.w_down"))
+                  self.W(p + "shared.w_down")) if s.ffn_shared else None
         if np.ndim(xn) == 1:
             return moe_ffn(xn, self.W(p + "router"), experts, shared, s.top_k)
         # diagnostic only: how close each row's routing came to a tie
@@ -248,8 +249,8 @@ class Decoder:
         srt = np.sort(logit)[::-1]
         self.route_gaps.append(float(srt[s.top_k - 1] - srt[s.top_k]))
         wsum = sum(r[e] for e in chosen)
-        y = swiglu_ffn(xn, self.W(p + "shared.w_gate"), self.W(p + "shared.w_up"),
-                       self.W(p + "shared.w_down"))
+        y = (swiglu_ffn(xn, self.W(p + "shared.w_gate"), self.W(p + "shared.w_up"),
+                        self.W(p + "shared.w_down")) if s.ffn_shared else np.zeros_like(xn))
         for e in chosen:
             q = p + f"experts.{e}."
             y = y + (r[e] / wsum) * swiglu_ffn(xn, self.W(q + "w_gate"),

@@ -123,10 +123,11 @@ def tensor_specs(s: Shape):
                 out += [(q + "w_gate", (s.ffn_expert, d), "w"),
                         (q + "w_up", (s.ffn_expert, d), "w"),
                         (q + "w_down", (d, s.ffn_expert), "w")]
-            q = p + "shared."
-            out += [(q + "w_gate", (s.ffn_shared, d), "w"),
-                    (q + "w_up", (s.ffn_shared, d), "w"),
-                    (q + "w_down", (d, s.ffn_shared), "w")]
+            if s.ffn_shared:  # Qwen-class MoE layers have no shared expert
+                q = p + "shared."
+                out += [(q + "w_gate", (s.ffn_shared, d), "w"),
+                        (q + "w_up", (s.ffn_shared, d), "w"),
+                        (q + "w_down", (d, s.ffn_shared), "w")]
         else:
             out += [(p + "w_gate", (s.ffn, d), "w"),
                     (p + "w_up", (s.ffn, d), "w"),

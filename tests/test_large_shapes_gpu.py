@@ -2,7 +2,8 @@
 the oracle through the C ABI: a 128,000-token vocabulary and a gate/up
 projection of 2 x 24,576 rows over 2,048 inputs (both run in row chunks; 3,460
 and 1,336 partial sums per CTA against 1,280), greedy and sampled; and 128
-routed experts with top-8."""
+routed experts with top-8; and 64 routed experts with top-8 and no shared
+expert (the layer of Mixtral- and OLMoE-class models)."""
 import numpy as np
 import pytest
 
@@ -15,6 +16,9 @@ pytestmark = pytest.mark.gpu
 
 WIDE = S.Shape("wide-vocab-ffn", n_layers=1, d_model=2048, n_heads=16, n_kv_heads=8, head_dim=128,
                ffn=24576, vocab=128000, prompt_len=16, decode_len=12, max_ctx=48)
+MOE_NOSHARED = S.Shape("moe-64x-top8-noshared", n_layers=2, d_model=512, n_heads=8, n_kv_heads=2, head_dim=64,
+                       ffn=0, vocab=3000, n_experts=64, top_k=8, ffn_expert=128, ffn_shared=0,
+                       prompt_len=20, decode_len=24, max_ctx=48)
 MOE_WIDE = S.Shape("moe-128x-top8", n_layers=2, d_model=512, n_heads=8, n_kv_heads=2, head_dim=64,
                    ffn=0, vocab=3000, n_experts=128, top_k=8, ffn_expert=64, ffn_shared=256,
                    prompt_len=20, decode_len=24, max_ctx=48)
@@ -56,9 +60,9 @@ def test_sampling_over_a_chunked_lm_head(wide):
     assert compared >= 0.75 * n
 
 
-def test_moe_128_experts_top8():
+@pytest.mark.parametrize("s", [MOE_WIDE, MOE_NOSHARED], ids=lambda s: s.name)
+def test_moe_many_experts_top8(s):
     # router weights scaled up so that the routing decisions are far from ties
-    s = MOE_WIDE
     w = S.make_weights(s, seed=32, cache=False)
     for l in range(s.n_layers):
         w[f"layers.{l}.router"] = (w[f"layers.{l}.router"].astype(np.float32) * 8).astype(np.float16)
@@ -77,4 +81,4 @@ def test_moe_128_experts_top8():
     bad = (max_abs > 2e-2) | (rel > 1e-3)
     assert not (bad & ~near).any(), np.flatnonzero(bad & ~near)
     assert bad.sum() <= 2
-    check_tokens(np.asarray(r["tokens"])[~bad], ol[~bad], "128 experts top-8")
+    check_tokens(np.asarray(r["tokens"])[~bad], ol[~bad], s.name)

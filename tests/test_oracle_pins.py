@@ -254,6 +254,10 @@ def _tiny(kind):
     if kind == "gqa":
         return S.Shape("t-gqa", n_layers=2, d_model=40, n_heads=5, n_kv_heads=2, head_dim=8,
                        ffn=24, vocab=53, max_ctx=24)
+    if kind == "moe-noshared":
+        return S.Shape("t-moe-ns", n_layers=2, d_model=32, n_heads=4, n_kv_heads=2, head_dim=8,
+                       ffn=0, vocab=47, n_experts=8, top_k=3, ffn_expert=16, ffn_shared=0,
+                       max_ctx=24)
     return S.Shape("t-moe", n_layers=2, d_model=32, n_heads=4, n_kv_heads=2, head_dim=8,
                    ffn=0, vocab=47, n_experts=6, top_k=2, ffn_expert=16, ffn_shared=24,
                    max_ctx=24)
@@ -264,7 +268,7 @@ def _scaled(w, k=10.0):
     return {n: (a * k).astype(np.float16) if a.ndim == 2 else a for n, a in w.items()}
 
 
-@pytest.mark.parametrize("kind", ["mha", "gqa", "moe"])
+@pytest.mark.parametrize("kind", ["mha", "gqa", "moe", "moe-noshared"])
 def test_incremental_decode_equals_full_recompute(kind):
     s = _tiny(kind)
     w = _scaled(S.make_weights(s, seed=3, cache=False))
@@ -467,3 +471,22 @@ def test_rope_wiring_in_the_model_brute_force(hk):
         for g in range(hk):
             assert list(cache["K"][0, g, j]) == Kc[j][g]
             assert list(cache["V"][0, g, j]) == Vc[j][g]
+
+
+def test_moe_without_shared_expert_equals_a_zero_shared_expert():
+    """A MoE layer with no shared expert (ffn_shared = 0, no shared tensors)
+    is the same function as one whose shared expert has all-zero weights:
+    SwiGLU of zero weights is zero, whatever the input."""
+    ns = _tiny("moe-noshared")
+    zs = ns.with_(name="t-moe-zero-shared", ffn_shared=8)
+    w = _scaled(S.make_weights(ns, seed=11, cache=False))
+    assert not any(".shared." in n for n in w)
+    wz = dict(w)
+    for l in range(zs.n_layers):
+        wz[f"layers.{l}.shared.w_gate"] = np.zeros((8, zs.d_model), np.float16)
+        wz[f"layers.{l}.shared.w_up"] = np.zeros((8, zs.d_model), np.float16)
+        wz[f"layers.{l}.shared.w_down"] = np.zeros((zs.d_model, 8), np.float16)
+    toks = S.make_tokens(ns, 12, seed=12)
+    a = O.Decoder(ns, w).forward_sequence(toks)
+    b = O.Decoder(zs, wz).forward_sequence(toks)
+    assert np.array_equal(a, b)

@@ -445,7 +445,7 @@ kie_status validate_config(const kie_config& k) {
   }
   if (moe) {
     if (k.ffn != 0 || k.top_k < 1 || k.top_k > kMaxTopK || k.top_k > k.n_experts ||
-        k.n_experts > kMaxExperts || k.ffn_expert < 8 || k.ffn_shared < 8 || k.ffn_expert % 8 ||
+        k.n_experts > kMaxExperts || k.ffn_expert < 8 || k.ffn_expert % 8 || k.ffn_shared < 0 ||
         k.ffn_shared % 8)
       return fail(nullptr, KIE_ERR_INVALID_ARG, "bad MoE shape");
   } else {
@@ -798,9 +798,11 @@ kie_status kie_load_weights(kie_ctx* c, const kie_tensor* tensors, int n, void* 
         W(q + "w_up", k.ffn_expert, d);
         W(q + "w_down", d, k.ffn_expert);
       }
-      W(p + "shared.w_gate", k.ffn_shared, d);
-      W(p + "shared.w_up", k.ffn_shared, d);
-      W(p + "shared.w_down", d, k.ffn_shared);
+      if (k.ffn_shared) {  // a model without a shared expert has no shared tensors
+        W(p + "shared.w_gate", k.ffn_shared, d);
+        W(p + "shared.w_up", k.ffn_shared, d);
+        W(p + "shared.w_down", d, k.ffn_shared);
+      }
     }
   }
   std::map<std::string, Tensor> got;
