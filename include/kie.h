@@ -59,8 +59,10 @@ typedef enum {
  * passed to kie_load_weights). Each expert's rows are split over all CTAs, so
  * every routing decision loads every SM with the same bytes.
  * Constraints: d_model, n_heads*head_dim, ffn, ffn_expert, ffn_shared multiples
- * of 8; head_dim 64 or 128; each KV head serves 1 to 4 query heads (query
- * head h reads KV head floor(h * n_kv_heads / n_heads)); max_ctx >= 1.
+ * of 8; head_dim 64 or 128; each KV head serves 1 to 16 query heads (query
+ * head h reads KV head floor(h * n_kv_heads / n_heads)), attended in equal
+ * sub-units of at most 4 (a shape whose uneven groups would leave a sub-unit
+ * empty is rejected); max_ctx >= 1.
  * Capacity of one launch (one CTA per SM, S SMs): the rows of every matrix are
  * split over the CTAs; a CTA keeps at most 64 residual rows (d_model <= 64 S,
  * checked by kie_create) and at most 1280 partial sums per phase (its rows of

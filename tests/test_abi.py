@@ -64,7 +64,7 @@ def _cfg(**kw):
 
 
 @pytest.mark.parametrize("bad", [dict(d_model=100), dict(head_dim=96), dict(n_kv_heads=8),
-                                 dict(n_heads=10, n_kv_heads=2), dict(max_ctx=0),
+                                 dict(n_heads=40, n_kv_heads=2), dict(max_ctx=0),
                                  dict(ffn=0), dict(n_experts=4, top_k=5, ffn=0, ffn_expert=64,
                                                    ffn_shared=64),
                                  dict(rope_theta=0.0)])

@@ -135,6 +135,24 @@ def test_gqa_long_context_multi_round_attention():
     check_tokens(gt, ol, "gqa-long")
 
 
+GQA_WIDE_SHORT = S.Shape("gqa-16:2", n_layers=2, d_model=1024, n_heads=16, n_kv_heads=2, head_dim=64,
+                         ffn=2048, vocab=4000, prompt_len=37, decode_len=40, max_ctx=80)
+GQA_WIDE_LONG = S.Shape("gqa-14:2-long", n_layers=2, d_model=896, n_heads=14, n_kv_heads=2, head_dim=64,
+                        ffn=1024, vocab=3000, prompt_len=2400, decode_len=24, max_ctx=2424)
+
+
+@pytest.mark.parametrize("s", [GQA_WIDE_SHORT, GQA_WIDE_LONG], ids=lambda s: s.name)
+def test_gqa_groups_wider_than_one_unit(s):
+    # more query heads per KV head than one attention unit holds (8:1 and 7:1):
+    # at short context every query head is its own unit; at ~2400 positions
+    # (11 chunks per head) each group runs as sub-units of 4 and 3 query heads
+    # over the same K/V rows, with cross-CTA chunk merges
+    w = S.make_weights(s, seed=9, cache=False)
+    gl, ol, gt, _ = forced_sequence_case(s, 9, s.decode_len, prompt_len=s.prompt_len, weights=w)
+    check_step_logits(gl, ol, s.name)
+    check_tokens(gt, ol, s.name)
+
+
 def test_long_context_full_size_self_consistency():
     # The long-context workload at full size (32768-token prompt, GQA 20:8, fp16
     # KV cache of 3.5 GB). The oracle cannot run a 32K-token 2.2B prefix, so the

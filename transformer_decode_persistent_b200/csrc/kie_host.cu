@@ -436,12 +436,19 @@ kie_status validate_config(const kie_config& k) {
     return fail(nullptr, KIE_ERR_INVALID_ARG, "head_dim must be 64 or 128");
   if (k.n_kv_heads > k.n_heads)
     return fail(nullptr, KIE_ERR_INVALID_ARG, "n_kv_heads > n_heads");
-  for (int g = 0; g < k.n_kv_heads; ++g) {
-    const int lo = (g * k.n_heads + k.n_kv_heads - 1) / k.n_kv_heads;
-    const int hi = ((g + 1) * k.n_heads + k.n_kv_heads - 1) / k.n_kv_heads;
-    if (hi - lo > kMaxHeadsPerGroup || hi - lo < 1)
-      return fail(nullptr, KIE_ERR_INVALID_ARG, "KV head %d serves %d query heads (1..%d allowed)", g,
-                  hi - lo, kMaxHeadsPerGroup);
+  // a KV head's query heads are attended in sub-units of at most
+  // kMaxHeadsPerGroup (the kernel's attention plan); every sub-unit needs one
+  {
+    const int gmax = (k.n_heads + k.n_kv_heads - 1) / k.n_kv_heads;
+    const int sub = (gmax + kMaxHeadsPerGroup - 1) / kMaxHeadsPerGroup, hs = (gmax + sub - 1) / sub;
+    for (int g = 0; g < k.n_kv_heads; ++g) {
+      const int lo = (g * k.n_heads + k.n_kv_heads - 1) / k.n_kv_heads;
+      const int hi = ((g + 1) * k.n_heads + k.n_kv_heads - 1) / k.n_kv_heads;
+      if (hi - lo < 1 || (sub - 1) * hs >= hi - lo || gmax > kMaxQueryHeadsPerKv)
+        return fail(nullptr, KIE_ERR_INVALID_ARG,
+                    "KV head %d serves %d query heads (1..%d allowed, in sub-units of at most %d)", g, hi - lo,
+                    kMaxQueryHeadsPerKv, kMaxHeadsPerGroup);
+    }
   }
   if (moe) {
     if (k.ffn != 0 || k.top_k < 1 || k.top_k > kMaxTopK || k.top_k > k.n_experts ||

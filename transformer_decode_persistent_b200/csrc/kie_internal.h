@@ -19,7 +19,8 @@ constexpr int kMaxStageBytes = 16384;                  // upper bound of one sta
 constexpr int kMaxRowsPerTile = 8;                     // rows of one tile in general (register-blocked)
 constexpr int kMaxRowsWide = 13;                       // rows of a tile 512 halves wide
 constexpr int kPartFloats = 1280;                      // per-CTA partial-sum slots per phase
-constexpr int kMaxHeadsPerGroup = 4;                   // query heads per KV head (GQA)
+constexpr int kMaxHeadsPerGroup = 4;                   // query heads of one attention unit
+constexpr int kMaxQueryHeadsPerKv = 16;                // query heads per KV head (GQA), in sub-units
 constexpr int kMaxTopK = 8;                            // routed experts per token
 constexpr int kAttnSub = 32;                           // positions per attention sub-block
 constexpr int kMaxExperts = 256;

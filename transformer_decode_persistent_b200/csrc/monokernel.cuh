@@ -434,14 +434,16 @@ static __device__ bool wait_bar(const Params& P, SmemCtl* sc, uint64_t* b, unsig
 // reads it directly.
 //
 // A unit is normally one KV head's chunk for all the query heads it serves
-// (its K/V rows are read once). When the query heads' units of every chunk
-// fit in one wave of CTAs (short context with grouped heads), each query head
-// becomes a unit of its own instead: the group's K/V rows are then read once
-// per query head, a small cost at short context, and the work of a group is
-// spread over as many CTAs as it has query heads. Per head the arithmetic and
-// its order are the same either way.
+// (its K/V rows are read once); a group of more than kMaxHeadsPerGroup query
+// heads is cut into `sub` equal sub-units of at most that many (each reads the
+// group's K/V rows). When the query heads' units of every chunk fit in one
+// wave of CTAs (short context with grouped heads), each query head becomes a
+// unit of its own instead: the group's K/V rows are then read once per query
+// head, a small cost at short context, and the work of a group is spread over
+// as many CTAs as it has query heads. Per head the arithmetic and its order
+// are the same either way.
 struct AttnPlan {
-  int T, per, pw, nsb, nchk, units, split;
+  int T, per, pw, nsb, nchk, units, split, sub, hs;
 };
 __device__ __forceinline__ AttnPlan attn_plan(int pos, int hk, int hq, int grid) {
   constexpr int kUnitMin = kConsumerWarps * kAttnSub;
@@ -454,12 +456,16 @@ __device__ __forceinline__ AttnPlan attn_plan(int pos, int hk, int hq, int grid)
   a.nsb = a.pw / kAttnSub;
   a.nchk = (a.T + per - 1) / per;
   a.split = (hq > hk && hq * a.nchk <= grid) ? 1 : 0;
-  a.units = (a.split ? hq : hk) * a.nchk;
+  const int gmax = (hq + hk - 1) / hk;  // query heads of the largest group
+  a.sub = (gmax + kMaxHeadsPerGroup - 1) / kMaxHeadsPerGroup;
+  a.hs = (gmax + a.sub - 1) / a.sub;
+  a.units = (a.split ? hq : hk * a.sub) * a.nchk;
   return a;
 }
 // Unit u: KV head g, chunk ch, query heads h_lo .. h_lo + nh - 1. KV head g
 // serves query heads ceil(g hq / hk) .. ceil((g + 1) hq / hk) - 1, so query
-// head q belongs to KV head floor(q hk / hq).
+// head q belongs to KV head floor(q hk / hq). The host admits only shapes in
+// which every sub-unit gets at least one query head.
 struct AttnUnit {
   int g, ch, h_lo, nh;
 };
@@ -472,9 +478,11 @@ __device__ __forceinline__ AttnUnit attn_unit(const AttnPlan& a, int u, int hk, 
     r.nh = 1;
     r.g = (int)(((long long)idx * hk) / hq);
   } else {
-    r.g = idx;
-    r.h_lo = (idx * hq + hk - 1) / hk;
-    r.nh = ((idx + 1) * hq + hk - 1) / hk - r.h_lo;
+    r.g = idx / a.sub;
+    const int sgi = idx - r.g * a.sub;
+    const int glo = (r.g * hq + hk - 1) / hk, ghi = ((r.g + 1) * hq + hk - 1) / hk;
+    r.h_lo = glo + sgi * a.hs;
+    r.nh = min(ghi, r.h_lo + a.hs) - r.h_lo;
   }
   return r;
 }
