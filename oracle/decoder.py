@@ -315,6 +315,25 @@ class Decoder:
         xn = rmsnorm(x, self.w16["final_norm"], s.rms_eps)
         return self.W("lm_head") @ xn
 
+    def fill_cache_one_layer(self, tokens, cache):
+        """For a one-layer model: the K/V cache of positions 0..T-1 straight
+        from ``tokens``, so a long prompt can be followed without T attention
+        steps. Layer 0's key and value at position p are the projections of the
+        normalised embedding of token p, rotated (the key) and rounded exactly
+        as ``step`` does; they need no attention output, and a one-layer model
+        caches nothing else. Advances the cache to position T."""
+        s = self.s
+        assert s.n_layers == 1 and cache["pos"] == 0
+        tokens = np.asarray(tokens)
+        T, dh = len(tokens), s.head_dim
+        xn = rmsnorm(f64(self.w16["embed"][tokens]), self.w16["layers.0.attn_norm"], s.rms_eps)
+        k = (xn @ self.W("layers.0.wk").T).reshape(T, s.n_kv_heads, dh)
+        v = (xn @ self.W("layers.0.wv").T).reshape(T, s.n_kv_heads, dh)
+        k = rope(k, np.arange(T), s.rope_theta)
+        cache["K"][0, :, :T, :] = self.kv(k).transpose(1, 0, 2)
+        cache["V"][0, :, :T, :] = self.kv(v).transpose(1, 0, 2)
+        cache["pos"] = T
+
     def greedy(self, prompt, n: int, forced=None, cache=None):
         """Greedy decode of ``n`` tokens after ``prompt``.
 

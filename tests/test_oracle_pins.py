@@ -490,3 +490,23 @@ def test_moe_without_shared_expert_equals_a_zero_shared_expert():
     a = O.Decoder(ns, w).forward_sequence(toks)
     b = O.Decoder(zs, wz).forward_sequence(toks)
     assert np.array_equal(a, b)
+
+
+def test_one_layer_cache_fill_equals_stepping_the_prompt():
+    """The one-layer cache fill (projections of the embedded prompt, for long
+    contexts) gives the same cache and the same following logits as
+    forwarding the prompt one token at a time."""
+    s = S.Shape("t-1l", n_layers=1, d_model=40, n_heads=5, n_kv_heads=2, head_dim=8,
+                ffn=24, vocab=53, max_ctx=40)
+    w = _scaled(S.make_weights(s, seed=21, cache=False))
+    toks = S.make_tokens(s, 30, seed=22)
+    a, b = O.Decoder(s, w), O.Decoder(s, w)
+    ca, cb = a.new_cache(40), b.new_cache(40)
+    for t in toks[:25]:
+        a.step(t, ca, want_logits=False)
+    b.fill_cache_one_layer(toks[:25], cb)
+    assert ca["pos"] == cb["pos"] == 25
+    assert np.allclose(ca["K"], cb["K"], rtol=0, atol=1e-12) and np.allclose(ca["V"], cb["V"], rtol=0, atol=1e-12)
+    for t in toks[25:]:
+        la, lb = a.step(t, ca), b.step(t, cb)
+        assert np.allclose(la, lb, rtol=0, atol=1e-10 * np.abs(la).max())

@@ -239,6 +239,33 @@ def test_dense_2b_benchmarked_run():
     assert np.array_equal(gm, srt[:, -1] - srt[:, -2])
 
 
+def test_long_context_32k_one_layer_oracle_parity():
+    # The long-context head layout (GQA 20:8, d 2560, head_dim 128) at the full
+    # 32768-token prompt, on one layer so that the oracle can follow: its
+    # cache comes from the prompt's projections (layer 0 needs no attention
+    # output for them), then 8 teacher-forced steps at positions 32767..32774
+    # compare logits with the engine's (tensor-core prompt path, then decode
+    # attention over ~32K positions in 19 chunks per head, more units than CTAs).
+    s = S.LONG_2B.with_(name="gqa20:8-32k-1L", n_layers=1, decode_len=8, max_ctx=32768 + 8)
+    w = S.make_weights(s, seed=4, cache=False)
+    prompt = S.make_prompt(s, 4)
+    cont = S.make_tokens(s, s.decode_len, 4)
+    P = len(prompt)
+    ref = O.Decoder(s, w)
+    cache = ref.new_cache(P + s.decode_len)
+    ref.fill_cache_one_layer(prompt[:-1], cache)
+    ol, cur = [], int(prompt[-1])
+    for i in range(s.decode_len):
+        ol.append(ref.step(cur, cache))
+        cur = int(cont[i])
+    ol = np.stack(ol)
+    eng = make_engine(s, w, max_ctx=P + s.decode_len)
+    eng.prefill(prompt)
+    r = eng.decode(s.decode_len, forced=cont.astype(np.int32), logits=True)
+    check_step_logits(r["logits"].cpu().numpy(), ol, "GQA 20:8, 32K context, one layer")
+    check_tokens(np.asarray(r["tokens"]), ol, "GQA 20:8, 32K context, one layer")
+
+
 def test_long_context_reduced_oracle_parity():
     # The long-context workload's weights and head layout (GQA 20:8 at d 2560)
     # with the prompt cut to 2048 tokens and 32 greedy steps, as far as the
