@@ -416,7 +416,7 @@ def main():
             torch.cuda.synchronize()
             pms.append(a.elapsed_time(b))
         prefill = {"prompt_tokens": P, "ms": min(pms), "tokens_per_s": (P - 1) / (min(pms) / 1000.0),
-                   "path": "tensor cores" if shape.n_experts == 0 else "decode kernel, forced tokens"}
+                   "path": "tensor cores"}
 
     stall = None
     if args.trace and rank == 0:

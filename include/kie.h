@@ -161,7 +161,9 @@ kie_status kie_create(const kie_config* cfg, int device, kie_ctx** out);
 /* Copy and pack the model weights into library-owned device memory (the
  * phase-ordered, per-CTA weight tape). The caller keeps ownership of its
  * buffers and may free them when the call returns. All tensors named in the
- * kie_tensor comment must be given exactly once with the stated shapes.
+ * kie_tensor comment must be given exactly once with the stated shapes. The
+ * library also keeps row-major copies of the layer matrices for the prompt
+ * path (about the model's size again in device memory).
  * May be called again to replace the weights; resets the position.
  * Errors: INVALID_ARG (missing/extra/misshapen tensor), CUDA, OOM. */
 kie_status kie_load_weights(kie_ctx* ctx, const kie_tensor* tensors, int n_tensors,
@@ -169,9 +171,12 @@ kie_status kie_load_weights(kie_ctx* ctx, const kie_tensor* tensors, int n_tenso
 
 /* Append `n` prompt tokens (host array, ids in [0, vocab)). Commits the pending
  * token (if any) and tokens[0..n-2] to the KV cache; tokens[n-1] becomes the
- * pending token. No logits are computed. One persistent launch.
+ * pending token. No logits are computed. The tokens run through the
+ * tensor-core prompt path in chunks of up to 1024 (tcgen05 GEMMs with fused
+ * epilogues, tensor-core attention over the cache; MoE: each routed expert
+ * over its own tokens).
  * Errors: STATE (no weights / poisoned), INVALID_ARG, CONTEXT_FULL, CUDA,
- * TIMEOUT. */
+ * TIMEOUT, DEVICE (a non-finite router logit). */
 kie_status kie_prefill(kie_ctx* ctx, const int32_t* tokens, int n, void* stream);
 
 /* Decode `n_tokens` tokens in ONE persistent launch. Step i forwards the pending

@@ -153,6 +153,42 @@ def test_gqa_groups_wider_than_one_unit(s):
     check_tokens(gt, ol, s.name)
 
 
+ZERO_DENSE = S.Shape("zero-dense", n_layers=2, d_model=512, n_heads=8, n_kv_heads=2, head_dim=64,
+                     ffn=1024, vocab=3000, prompt_len=9, decode_len=12, max_ctx=24)
+ZERO_MOE = S.Shape("zero-moe", n_layers=2, d_model=512, n_heads=8, n_kv_heads=2, head_dim=64, ffn=0,
+                   vocab=3000, n_experts=8, top_k=2, ffn_expert=128, ffn_shared=256, prompt_len=9,
+                   decode_len=12, max_ctx=24)
+
+
+@pytest.mark.parametrize("case", ["Z1-dense", "Z2-dense", "Z2-moe"])
+def test_zero_weight_closed_forms_on_the_gpu(case):
+    # Z1: every layer matrix zero; Z2: only the output and down projections
+    # (MoE: every expert's and the shared expert's) zero. Either way each
+    # block adds nothing to the residual stream, whatever attention and the
+    # FFN compute, so the logits of every step are lm_head . RMSNorm(E[t]; g_f)
+    # of the step's input token t: a closed form written out here in numpy,
+    # independent of the oracle. Isolates GEMV / LM-head errors from
+    # attention and routing.
+    s = ZERO_MOE if case.endswith("moe") else ZERO_DENSE
+    w = S.make_weights(s, seed=13, cache=False)
+    for n in list(w):
+        if not n.startswith("layers.") or w[n].ndim != 2:
+            continue
+        if case.startswith("Z1") or n.endswith(".wo") or n.endswith(".w_down"):
+            w[n] = np.zeros_like(w[n])
+    prompt = S.make_prompt(s, 13)
+    cont = S.make_tokens(s, s.decode_len, 13)
+    inputs = np.concatenate([prompt[-1:], cont[:-1]])  # the token each step forwards
+    e = w["embed"][inputs].astype(np.float64)
+    xn = e / np.sqrt((e * e).mean(axis=1, keepdims=True) + s.rms_eps) * w["final_norm"].astype(np.float64)
+    closed = xn @ w["lm_head"].astype(np.float64).T
+    eng = make_engine(s, w)
+    eng.prefill(prompt)
+    r = eng.decode(s.decode_len, forced=cont.astype(np.int32), logits=True)
+    check_step_logits(r["logits"].cpu().numpy(), closed, case)
+    check_tokens(np.asarray(r["tokens"]), closed, case)
+
+
 def test_long_context_full_size_self_consistency():
     # The long-context workload at full size (32768-token prompt, GQA 20:8, fp16
     # KV cache of 3.5 GB). The oracle cannot run a 32K-token 2.2B prefix, so the
@@ -186,12 +222,24 @@ def test_long_context_full_size_self_consistency():
     assert np.isfinite(lg).all() and (np.std(lg, axis=1) > 0.1).all()
 
 
-def test_prompt_path_matches_decode_path_and_oracle():
+MOE_PROMPT = S.Shape("moe-prompt", n_layers=3, d_model=1024, n_heads=8, n_kv_heads=2, head_dim=128, ffn=0,
+                     vocab=8000, n_experts=16, top_k=2, ffn_expert=512, ffn_shared=1024, prompt_len=300,
+                     decode_len=16, max_ctx=316)
+MOE_PROMPT_NS = S.Shape("moe-prompt-64x-top8-noshared", n_layers=2, d_model=512, n_heads=8, n_kv_heads=2,
+                        head_dim=64, ffn=0, vocab=3000, n_experts=64, top_k=8, ffn_expert=128, ffn_shared=0,
+                        prompt_len=300, decode_len=16, max_ctx=316)
+
+
+@pytest.mark.parametrize("s", [S.SMALL, MOE_PROMPT, MOE_PROMPT_NS], ids=lambda s: s.name)
+def test_prompt_path_matches_decode_path_and_oracle(s):
     # The tensor-core prompt path and the decode kernel run teacher-forced over
     # the same prompt fill caches whose next 16 steps agree with each other and
-    # with the oracle under the parity criteria.
-    s = S.SMALL
-    w = S.make_weights(s, seed=0)
+    # with the oracle under the parity criteria. MoE: the prompt path routes
+    # each chunk (router GEMM, top-k, experts over their own sorted rows); the
+    # router weights are scaled up so that no routing decision is near a tie.
+    w = S.make_weights(s, seed=0, cache=not s.n_experts)
+    for l in range(s.n_layers if s.n_experts else 0):
+        w[f"layers.{l}.router"] = (w[f"layers.{l}.router"].astype(np.float32) * 8).astype(np.float16)
     prompt = S.make_prompt(s, 0)
     P = len(prompt)
     eng = make_engine(s, w, max_ctx=P + 16)

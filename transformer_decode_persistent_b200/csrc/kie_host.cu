@@ -90,11 +90,24 @@ struct kie_ctx {
   int64_t launches = 0;
   int64_t stream_bytes = 0;
   std::string err;
-  // tensor-core prompt prefill (dense models): row-major layer matrices in
-  // the packed row orders (q/k/v RoPE pairs and gate/up pairs adjacent),
-  // activation buffers for one chunk, and their tensor maps
+  // tensor-core prompt prefill: row-major layer matrices in the packed row
+  // orders (q/k/v RoPE pairs and gate/up pairs adjacent), activation buffers
+  // for one chunk, and their tensor maps
   bool pf_ready = false;
-  __half *pf_w[4] = {nullptr, nullptr, nullptr, nullptr};  // [L][rows][K]: q/k/v, o, gate/up, down
+  // [L][rows][K]: q/k/v, o, gate/up, down (MoE: the shared expert's gate/up and down)
+  __half *pf_w[4] = {nullptr, nullptr, nullptr, nullptr};
+  // MoE: the routed experts' [L][E][rows][K] gate/up and down, the router
+  // [L][E rounded up to a GEMM tile][d] (zero rows past E), routing buffers,
+  // the expert-sorted activations and hidden rows, the experts' outputs
+  __half *pf_we[2] = {nullptr, nullptr};
+  __half* pf_router = nullptr;
+  int pf_epad = 0;
+  float *pf_logits = nullptr, *pf_wt = nullptr, *pf_y = nullptr;
+  int *pf_sel = nullptr, *pf_range = nullptr, *pf_rowof = nullptr, *pf_tokof = nullptr;
+  __half *pf_gh = nullptr, *pf_gl = nullptr, *pf_eh = nullptr, *pf_el = nullptr;
+  std::vector<CUtensorMap> pf_emap;  // [L][E][2]
+  std::vector<CUtensorMap> pf_rmap;  // [L]
+  CUtensorMap pf_map_gh{}, pf_map_gl{}, pf_map_eh{}, pf_map_el{};
   float *pf_x = nullptr, *pf_q = nullptr;
   __half *pf_xh = nullptr, *pf_xl = nullptr, *pf_oh = nullptr, *pf_ol = nullptr, *pf_hh = nullptr, *pf_hl = nullptr;
   int *pf_tok = nullptr, *pf_err = nullptr;
@@ -467,19 +480,37 @@ kie_status validate_config(const kie_config& k) {
 
 }  // namespace
 
-// Buffers and tensor maps of the tensor-core prefill (dense models), once the
-// prefill weights exist.
+// Buffers and tensor maps of the tensor-core prefill, once the prefill weights
+// exist. `ff` is the dense FFN width, or the MoE shared expert's (0: none).
 static kie_status prefill_setup(kie_ctx* c) {
   using namespace kie::pf;
   const kie_config& k = c->cfg;
-  const int d = k.d_model, hq = k.n_heads, hk = k.n_kv_heads, dh = k.head_dim, L = k.n_layers, ff = k.ffn;
+  const bool moe = k.n_experts > 0;
+  const int d = k.d_model, hq = k.n_heads, hk = k.n_kv_heads, dh = k.head_dim, L = k.n_layers;
+  const int ff = moe ? k.ffn_shared : k.ffn, E = k.n_experts, ffe = k.ffn_expert, rows = kChunk * k.top_k;
   kie_status s;
+  if (moe && !c->pf_logits) {
+    if ((s = dalloc(c, &c->pf_logits, (size_t)kChunk * E * 4)) || (s = dalloc(c, &c->pf_wt, (size_t)rows * 4)) ||
+        (s = dalloc(c, &c->pf_y, (size_t)rows * d * 4)) || (s = dalloc(c, &c->pf_sel, (size_t)rows * 4)) ||
+        (s = dalloc(c, &c->pf_range, (size_t)E * 2 * 4)) || (s = dalloc(c, &c->pf_rowof, (size_t)rows * 4)) ||
+        (s = dalloc(c, &c->pf_tokof, (size_t)rows * 4)) || (s = dalloc(c, &c->pf_gh, (size_t)rows * d * 2)) ||
+        (s = dalloc(c, &c->pf_gl, (size_t)rows * d * 2)) || (s = dalloc(c, &c->pf_eh, (size_t)rows * ffe * 2)) ||
+        (s = dalloc(c, &c->pf_el, (size_t)rows * ffe * 2)))
+      return s;
+    // rows past an expert's range are read by its last GEMM tile (their
+    // columns are discarded); keep them finite
+    CUDA_TRY(c, cudaMemset(c->pf_gh, 0, (size_t)rows * d * 2));
+    CUDA_TRY(c, cudaMemset(c->pf_gl, 0, (size_t)rows * d * 2));
+    CUDA_TRY(c, cudaMemset(c->pf_eh, 0, (size_t)rows * ffe * 2));
+    CUDA_TRY(c, cudaMemset(c->pf_el, 0, (size_t)rows * ffe * 2));
+  }
   if (!c->pf_x) {
     if ((s = dalloc(c, &c->pf_x, (size_t)kChunk * d * 4)) || (s = dalloc(c, &c->pf_q, (size_t)kChunk * hq * dh * 4)) ||
         (s = dalloc(c, &c->pf_xh, (size_t)kChunk * d * 2)) || (s = dalloc(c, &c->pf_xl, (size_t)kChunk * d * 2)) ||
         (s = dalloc(c, &c->pf_oh, (size_t)kChunk * hq * dh * 2)) ||
         (s = dalloc(c, &c->pf_ol, (size_t)kChunk * hq * dh * 2)) ||
-        (s = dalloc(c, &c->pf_hh, (size_t)kChunk * ff * 2)) || (s = dalloc(c, &c->pf_hl, (size_t)kChunk * ff * 2)) ||
+        (ff && (s = dalloc(c, &c->pf_hh, (size_t)kChunk * ff * 2))) ||
+        (ff && (s = dalloc(c, &c->pf_hl, (size_t)kChunk * ff * 2))) ||
         (s = dalloc(c, &c->pf_tok, (size_t)kChunk * 4)) || (s = dalloc(c, &c->pf_err, 16)))
       return s;
     // rows past a chunk's length are read by the last GEMM tile (their
@@ -488,20 +519,38 @@ static kie_status prefill_setup(kie_ctx* c) {
     CUDA_TRY(c, cudaMemset(c->pf_xl, 0, (size_t)kChunk * d * 2));
     CUDA_TRY(c, cudaMemset(c->pf_oh, 0, (size_t)kChunk * hq * dh * 2));
     CUDA_TRY(c, cudaMemset(c->pf_ol, 0, (size_t)kChunk * hq * dh * 2));
-    CUDA_TRY(c, cudaMemset(c->pf_hh, 0, (size_t)kChunk * ff * 2));
-    CUDA_TRY(c, cudaMemset(c->pf_hl, 0, (size_t)kChunk * ff * 2));
+    if (ff) {
+      CUDA_TRY(c, cudaMemset(c->pf_hh, 0, (size_t)kChunk * ff * 2));
+      CUDA_TRY(c, cudaMemset(c->pf_hl, 0, (size_t)kChunk * ff * 2));
+    }
     CUDA_TRY(c, cudaMemset(c->pf_err, 0, 16));
   }
   bool ok = make_map(&c->pf_map_xh, c->pf_xh, kChunk, d, kBN) && make_map(&c->pf_map_xl, c->pf_xl, kChunk, d, kBN) &&
             make_map(&c->pf_map_oh, c->pf_oh, kChunk, hq * dh, kBN) &&
             make_map(&c->pf_map_ol, c->pf_ol, kChunk, hq * dh, kBN) &&
-            make_map(&c->pf_map_hh, c->pf_hh, kChunk, ff, kBN) && make_map(&c->pf_map_hl, c->pf_hl, kChunk, ff, kBN);
+            (!ff || (make_map(&c->pf_map_hh, c->pf_hh, kChunk, ff, kBN) &&
+                     make_map(&c->pf_map_hl, c->pf_hl, kChunk, ff, kBN)));
   const int prow[4] = {(hq + 2 * hk) * dh, d, 2 * ff, d};
   const int pk[4] = {d, hq * dh, d, ff};
   c->pf_wmap.assign((size_t)L * 4, CUtensorMap{});
   for (int l = 0; l < L && ok; ++l)
     for (int m = 0; m < 4 && ok; ++m)
-      ok = make_map(&c->pf_wmap[(size_t)l * 4 + m], c->pf_w[m] + (size_t)l * prow[m] * pk[m], prow[m], pk[m], kBM);
+      if (m < 2 || ff)
+        ok = make_map(&c->pf_wmap[(size_t)l * 4 + m], c->pf_w[m] + (size_t)l * prow[m] * pk[m], prow[m], pk[m], kBM);
+  if (moe && ok) {
+    ok = make_map(&c->pf_map_gh, c->pf_gh, rows, d, kBN) && make_map(&c->pf_map_gl, c->pf_gl, rows, d, kBN) &&
+         make_map(&c->pf_map_eh, c->pf_eh, rows, ffe, kBN) && make_map(&c->pf_map_el, c->pf_el, rows, ffe, kBN);
+    c->pf_emap.assign((size_t)L * E * 2, CUtensorMap{});
+    c->pf_rmap.assign((size_t)L, CUtensorMap{});
+    for (int l = 0; l < L && ok; ++l) {
+      ok = make_map(&c->pf_rmap[l], c->pf_router + (size_t)l * c->pf_epad * d, c->pf_epad, d, kBM);
+      for (int e = 0; e < E && ok; ++e) {
+        const size_t ge = (size_t)l * E + e;
+        ok = make_map(&c->pf_emap[ge * 2], c->pf_we[0] + ge * 2 * ffe * d, 2 * ffe, d, kBM) &&
+             make_map(&c->pf_emap[ge * 2 + 1], c->pf_we[1] + ge * d * ffe, d, ffe, kBM);
+      }
+    }
+  }
   if (!ok) return fail(c, KIE_ERR_CUDA, "tensor map encoding for the prefill failed");
   c->pf_ready = true;
   return KIE_OK;
@@ -513,7 +562,9 @@ static kie_status prefill_setup(kie_ctx* c) {
 static kie_status prefill_tc(kie_ctx* c, const std::vector<int32_t>& seq, cudaStream_t st) {
   using namespace kie::pf;
   const kie_config& k = c->cfg;
-  const int d = k.d_model, hq = k.n_heads, hk = k.n_kv_heads, dh = k.head_dim, L = k.n_layers, ff = k.ffn;
+  const bool moe = k.n_experts > 0;
+  const int d = k.d_model, hq = k.n_heads, hk = k.n_kv_heads, dh = k.head_dim, L = k.n_layers;
+  const int ff = moe ? k.ffn_shared : k.ffn, E = k.n_experts, ffe = k.ffn_expert, K = k.top_k;
   const int qkv_rows = (hq + 2 * hk) * dh;
   CUDA_TRY(c, cudaMemsetAsync(c->pf_err, 0, 4, st));
   for (size_t c0 = 0; c0 < seq.size(); c0 += kChunk) {
@@ -539,15 +590,52 @@ static kie_status prefill_tc(kie_ctx* c, const std::vector<int32_t>& seq, cudaSt
       o.M = d; o.N = T; o.K = hq * dh; o.epi = EPI_RESID; o.x = c->pf_x;
       CUDA_TRY(c, gemm(W[1], c->pf_map_oh, c->pf_map_ol, o, st));
       CUDA_TRY(c, rmsnorm_split(c->pf_x, c->mlp_norm + (size_t)l * d, c->pf_xh, c->pf_xl, T, d, k.rms_eps, st));
-      GemmArgs u{};
-      u.err = c->pf_err;
-      u.M = 2 * ff; u.N = T; u.K = d; u.epi = EPI_SWIGLU; u.h_hi = c->pf_hh; u.h_lo = c->pf_hl; u.ff = ff;
-      CUDA_TRY(c, gemm(W[2], c->pf_map_xh, c->pf_map_xl, u, st));
-      GemmArgs w{};
-      w.err = c->pf_err;
-      w.M = d; w.N = T; w.K = ff; w.epi = EPI_RESID; w.x = c->pf_x;
-      CUDA_TRY(c, gemm(W[3], c->pf_map_hh, c->pf_map_hl, w, st));
-      c->launches += 5;
+      if (moe) {
+        // router logits, routing and the expert-sorted rows, then each routed
+        // expert over its own rows, the shared expert over all, and the
+        // weighted combine into x
+        GemmArgs r{};
+        r.err = c->pf_err;
+        r.M = E; r.N = T; r.K = d; r.epi = EPI_STORE; r.out = c->pf_logits;
+        CUDA_TRY(c, gemm(c->pf_rmap[l], c->pf_map_xh, c->pf_map_xl, r, st));
+        RouteArgs ra{c->pf_logits, c->pf_sel, c->pf_wt, c->pf_range, c->pf_rowof, c->pf_tokof, c->pf_err, T, E, K};
+        CUDA_TRY(c, moe_route(ra, st));
+        CUDA_TRY(c, moe_gather(c->pf_tokof, c->pf_xh, c->pf_xl, c->pf_gh, c->pf_gl, T * K, d, st));
+        for (int e = 0; e < E; ++e) {
+          const CUtensorMap* We = &c->pf_emap[((size_t)l * E + e) * 2];
+          GemmArgs u{};
+          u.err = c->pf_err;
+          u.M = 2 * ffe; u.N = T; u.K = d; u.epi = EPI_SWIGLU; u.h_hi = c->pf_eh; u.h_lo = c->pf_el; u.ff = ffe;
+          u.nrange = c->pf_range + 2 * e;
+          CUDA_TRY(c, gemm(We[0], c->pf_map_gh, c->pf_map_gl, u, st));
+          GemmArgs w{};
+          w.err = c->pf_err;
+          w.M = d; w.N = T; w.K = ffe; w.epi = EPI_STORE; w.out = c->pf_y; w.nrange = c->pf_range + 2 * e;
+          CUDA_TRY(c, gemm(We[1], c->pf_map_eh, c->pf_map_el, w, st));
+        }
+        if (ff) {
+          GemmArgs u{};
+          u.err = c->pf_err;
+          u.M = 2 * ff; u.N = T; u.K = d; u.epi = EPI_SWIGLU; u.h_hi = c->pf_hh; u.h_lo = c->pf_hl; u.ff = ff;
+          CUDA_TRY(c, gemm(W[2], c->pf_map_xh, c->pf_map_xl, u, st));
+          GemmArgs w{};
+          w.err = c->pf_err;
+          w.M = d; w.N = T; w.K = ff; w.epi = EPI_RESID; w.x = c->pf_x;
+          CUDA_TRY(c, gemm(W[3], c->pf_map_hh, c->pf_map_hl, w, st));
+        }
+        CUDA_TRY(c, moe_combine(c->pf_y, c->pf_rowof, c->pf_wt, c->pf_x, T, K, d, st));
+        c->launches += 7 + 2 * E + (ff ? 2 : 0);
+      } else {
+        GemmArgs u{};
+        u.err = c->pf_err;
+        u.M = 2 * ff; u.N = T; u.K = d; u.epi = EPI_SWIGLU; u.h_hi = c->pf_hh; u.h_lo = c->pf_hl; u.ff = ff;
+        CUDA_TRY(c, gemm(W[2], c->pf_map_xh, c->pf_map_xl, u, st));
+        GemmArgs w{};
+        w.err = c->pf_err;
+        w.M = d; w.N = T; w.K = ff; w.epi = EPI_RESID; w.x = c->pf_x;
+        CUDA_TRY(c, gemm(W[3], c->pf_map_hh, c->pf_map_hl, w, st));
+        c->launches += 5;
+      }
     }
     c->launches += 1;
   }
@@ -560,6 +648,7 @@ static kie_status prefill_tc(kie_ctx* c, const std::vector<int32_t>& seq, cudaSt
   CUDA_TRY(c, cudaMemcpy(&err, c->pf_err, 4, cudaMemcpyDeviceToHost));
   if (err) {
     c->poisoned = true;
+    if (err == 2) return fail(c, KIE_ERR_DEVICE, "prefill routing met a non-finite router logit; context poisoned");
     return fail(c, KIE_ERR_TIMEOUT, "prefill GEMM wait gave up; context poisoned");
   }
   return KIE_OK;
@@ -985,13 +1074,19 @@ kie_status kie_load_weights(kie_ctx* c, const kie_tensor* tensors, int n, void* 
     dfree(c, staging);
     return ps;
   }
-  // the prefill's row-major copies of the layer matrices (dense models)
+  // the prefill's row-major copies of the layer matrices in the packed row
+  // orders (slots 0-3: q/k/v, o, and the dense or shared-expert gate/up and
+  // down; MoE: the routed experts and the router as well)
   for (int i = 0; i < 4; ++i) { dfree(c, c->pf_w[i]); c->pf_w[i] = nullptr; }
+  for (int i = 0; i < 2; ++i) { dfree(c, c->pf_we[i]); c->pf_we[i] = nullptr; }
+  dfree(c, c->pf_router); c->pf_router = nullptr;
   c->pf_ready = false;
-  if (!moe) {
-    const int prow[4] = {(hq + 2 * hk) * dh, d, 2 * k.ffn, d};
-    const int pk[4] = {d, hq * dh, d, k.ffn};
+  {
+    const int fw = moe ? ffs : k.ffn;
+    const int prow[4] = {(hq + 2 * hk) * dh, d, 2 * fw, d};
+    const int pk[4] = {d, hq * dh, d, fw};
     for (int m = 0; m < 4 && ps == KIE_OK; ++m) {
+      if (m >= 2 && fw == 0) break;  // no shared expert
       if ((ps = dalloc(c, &c->pf_w[m], (size_t)L * prow[m] * pk[m] * 2))) break;
       for (int l = 0; l < L && ps == KIE_OK; ++l) {
         for (int r = 0; r < prow[m]; ++r) {
@@ -1000,6 +1095,31 @@ kie_status kie_load_weights(kie_ctx* c, const kie_tensor* tensors, int n, void* 
           hn.push_back(pk[m] / 8);
         }
         ps = flush();
+      }
+    }
+    if (moe && ps == KIE_OK) {
+      const int E = k.n_experts;
+      const int erow[2] = {2 * ffe, d}, ek[2] = {d, ffe};
+      for (int m = 0; m < 2 && ps == KIE_OK; ++m) {
+        if ((ps = dalloc(c, &c->pf_we[m], (size_t)L * E * erow[m] * ek[m] * 2))) break;
+        for (int l = 0; l < L && ps == KIE_OK; ++l) {
+          for (int e = 0; e < E; ++e)
+            for (int r = 0; r < erow[m]; ++r) {
+              hsrc.push_back((unsigned long long)rowptr(l, 4 + m * E + e, r));
+              hdst.push_back((unsigned long long)(c->pf_we[m] + (((size_t)l * E + e) * erow[m] + r) * ek[m]));
+              hn.push_back(ek[m] / 8);
+            }
+          ps = flush();
+        }
+      }
+      // the router, zero rows past E up to a whole GEMM tile
+      c->pf_epad = (E + kie::pf::kBM - 1) / kie::pf::kBM * kie::pf::kBM;
+      if (ps == KIE_OK && (ps = dalloc(c, &c->pf_router, (size_t)L * c->pf_epad * d * 2)) == KIE_OK) {
+        CUDA_TRY(c, cudaMemsetAsync(c->pf_router, 0, (size_t)L * c->pf_epad * d * 2, st));
+        for (int l = 0; l < L; ++l)
+          CUDA_TRY(c, cudaMemcpyAsync(c->pf_router + (size_t)l * c->pf_epad * d,
+                                      dptr["layers." + std::to_string(l) + ".router"], (size_t)E * d * 2,
+                                      cudaMemcpyDeviceToDevice, st));
       }
     }
     if (ps != KIE_OK) {
@@ -1046,7 +1166,7 @@ kie_status kie_load_weights(kie_ctx* c, const kie_tensor* tensors, int n, void* 
   }
   sb += (int64_t)k.vocab * d * 2 + (2LL * L + 1) * d * 2 + (int64_t)d * 2;
   c->stream_bytes = sb;
-  if (!moe) {
+  {
     kie_status s2 = prefill_setup(c);
     if (s2 != KIE_OK) return s2;
   }
@@ -1179,35 +1299,14 @@ kie_status kie_prefill(kie_ctx* c, const int32_t* tokens, int n, void* stream) {
   cudaStream_t st = (cudaStream_t)stream;
   const int32_t new_pending = tokens[n - 1];
   const int32_t pos_before = c->pos, pend_before = c->pending;
-  if (c->pf_ready) {
-    // dense models: the chunked tensor-core prefill
-    kie_status s = prefill_tc(c, seq, st);
-    if (s != KIE_OK) {
-      if (!c->poisoned) { c->pos = pos_before; c->pending = pend_before; }
-      return s;
-    }
-    c->pos += (int32_t)seq.size();
-    c->pending = new_pending;
-    return KIE_OK;
+  if (!c->pf_ready) return fail(c, KIE_ERR_STATE, "the prompt path is not set up (load weights first)");
+  // the chunked tensor-core prefill
+  kie_status s = prefill_tc(c, seq, st);
+  if (s != KIE_OK) {
+    if (!c->poisoned) { c->pos = pos_before; c->pending = pend_before; }
+    return s;
   }
-  // MoE models: the decode kernel in forced-token mode, one position per step
-  const int kChunk = 8192;  // bounds the barrier counter and the flag epochs of one launch
-  size_t i0 = 0;
-  while (i0 < seq.size()) {
-    const int m = (int)std::min<size_t>(kChunk, seq.size() - i0);
-    // forced[i] = token fed after step i
-    std::vector<int32_t> f(m);
-    for (int i = 0; i < m; ++i) f[i] = (i0 + i + 1 < seq.size()) ? seq[i0 + i + 1] : new_pending;
-    CUDA_TRY(c, cudaMemcpyAsync(c->forced_dev, f.data(), (size_t)m * 4, cudaMemcpyHostToDevice, st));
-    Run r{seq[i0], m, m, c->forced_dev, c->tok_dev, nullptr, nullptr, 0, -1, -1, nullptr, 0};
-    kie_status s = launch(c, r, st);
-    if (s != KIE_OK) {
-      if (!c->poisoned) { c->pos = pos_before; c->pending = pend_before; }
-      return s;
-    }
-    c->pos += m;
-    i0 += m;
-  }
+  c->pos += (int32_t)seq.size();
   c->pending = new_pending;
   return KIE_OK;
 }

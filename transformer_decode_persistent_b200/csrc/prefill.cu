@@ -120,15 +120,24 @@ __device__ __forceinline__ void split_store(__half* hi, __half* lo, size_t i, fl
 
 // Epilogue for one 32-token slice of the accumulator: this thread holds
 // D[row][n .. n+32) (row = this thread's weight row). Rows beyond M and
-// tokens beyond N are skipped; the lane-pair exchanges run on every lane.
-__device__ __forceinline__ void epilogue(const GemmArgs& a, int row, int n, const float (&v)[32]) {
+// tokens beyond N are skipped; the lane-pair exchanges run on every lane. tb
+// is the first token row of a device-resident range (0 otherwise): output
+// rows are tb + n + j.
+__device__ __forceinline__ void epilogue(const GemmArgs& a, int row, int tb, int n, int N, const float (&v)[32]) {
   const int lane = threadIdx.x & 31;
   const bool row_ok = row < a.M;
   if (a.epi == EPI_RESID) {
     if (!row_ok) return;
 #pragma unroll 4
     for (int j = 0; j < 32; ++j)
-      if (n + j < a.N) a.x[(size_t)(n + j) * a.M + row] += v[j];
+      if (n + j < N) a.x[(size_t)(tb + n + j) * a.M + row] += v[j];
+    return;
+  }
+  if (a.epi == EPI_STORE) {
+    if (!row_ok) return;
+#pragma unroll 4
+    for (int j = 0; j < 32; ++j)
+      if (n + j < N) a.out[(size_t)(tb + n + j) * a.M + row] = v[j];
     return;
   }
   if (a.epi == EPI_SWIGLU) {
@@ -136,9 +145,9 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, int row, int n, cons
 #pragma unroll 4
     for (int j = 0; j < 32; ++j) {
       const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
-      if (row_ok && !(lane & 1) && n + j < a.N) {
+      if (row_ok && !(lane & 1) && n + j < N) {
         const float h = silu(v[j]) * other;
-        split_store(a.h_hi, a.h_lo, (size_t)(n + j) * a.ff + row / 2, h);
+        split_store(a.h_hi, a.h_lo, (size_t)(tb + n + j) * a.ff + row / 2, h);
       }
     }
     return;
@@ -152,7 +161,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, int row, int n, cons
   for (int j = 0; j < 32; ++j) {
     const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
     const int t = n + j;
-    if (!row_ok || t >= a.N) continue;
+    if (!row_ok || t >= N) continue;
     const int pos = a.pos0 + t;
     if (H < a.hq + a.hk) {
       const float2 cs = a.rope[(size_t)pos * (dh / 2) + pi];
@@ -181,6 +190,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * kBM, n0 = blockIdx.y * kBN;
   const int nkb = (a.K + kBK - 1) / kBK;
+  // tokens: B rows tb .. tb + N - 1 (a device-resident range, or 0 .. a.N - 1)
+  int tb = 0, N = a.N;
+  if (a.nrange) {
+    tb = a.nrange[0];
+    N = min(a.N, a.nrange[1]);
+  }
+  if (n0 >= N) return;  // the whole CTA: before any barrier or tensor-memory allocation
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(&full[s])));
@@ -213,8 +229,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(&full[s])), "r"(kStageBytes)
                    : "memory");
       tma2d(su32(st), &tmA, kb * kBK, m0, su32(&full[s]));
-      tma2d(su32(st + kTileA), &tmBh, kb * kBK, n0, su32(&full[s]));
-      tma2d(su32(st + kTileA + kTileB), &tmBl, kb * kBK, n0, su32(&full[s]));
+      tma2d(su32(st + kTileA), &tmBh, kb * kBK, tb + n0, su32(&full[s]));
+      tma2d(su32(st + kTileA + kTileB), &tmBl, kb * kBK, tb + n0, su32(&full[s]));
     }
     // let every copy this thread issued land before the CTA can exit (on the
     // normal path the MMA issuer has already waited for all of them)
@@ -248,7 +264,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int c = 0; c < kBN; c += 32) {
       float v[32];
       tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
-      if (n0 + c < a.N) epilogue(a, row, n0 + c, v);
+      if (n0 + c < N) epilogue(a, row, tb, n0 + c, N, v);
     }
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -281,6 +297,126 @@ __global__ void rmsnorm_split_kernel(const float* x, const __half* g, __half* hi
   for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += red[w];
   const float inv = 1.0f / sqrtf(tot / (float)d + eps);
   for (int i = threadIdx.x; i < d; i += blockDim.x) split_store(hi, lo, (size_t)t * d + i, xr[i] * inv * __half2float(g[i]));
+}
+
+// ---------------------------------------------------------------- MoE routing
+
+constexpr int kRouteThreads = 1024;
+constexpr int kRoutePerLane = 8;  // experts a lane holds: up to 256 experts
+
+// One block for the whole chunk. (1) Warp w routes tokens w, w + 32, ...: the
+// softmax numerators of the token's router logits (the denominator cancels in
+// the renormalisation), top_k rounds of a warp arg-max with the lower expert
+// index on ties, weights renormalised over the chosen. (2) Warp w counts and
+// ranks the (token, slot) pairs of experts w, w + 32, ... in pair order
+// (ballots), so the sorted order is the pair order within each expert. (3)
+// Offsets and each pair's row in the expert-sorted order.
+__global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(RouteArgs a) {
+  extern __shared__ int sm_route[];
+  int* rank = sm_route;                     // [T * top_k]
+  int* off = rank + a.T * a.top_k;          // [E]
+  int* cnt = off + a.E;                     // [E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = kRouteThreads / 32;
+  const int P = a.T * a.top_k;
+  for (int t = warp; t < a.T; t += nw) {
+    const float* lg = a.logits + (size_t)t * a.E;
+    float pr[kRoutePerLane];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kRoutePerLane; ++i) {
+      const int e = lane + 32 * i;
+      pr[i] = e < a.E ? lg[e] : -INFINITY;
+      mx = fmaxf(mx, pr[i]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+#pragma unroll
+    for (int i = 0; i < kRoutePerLane; ++i) pr[i] = (lane + 32 * i < a.E) ? expf(pr[i] - mx) : -1.f;
+    float wsum = 0.f;
+    for (int k = 0; k < a.top_k; ++k) {
+      float bv = -1.f;
+      int bi = INT_MAX;
+#pragma unroll
+      for (int i = 0; i < kRoutePerLane; ++i)
+        if (pr[i] > bv) {
+          bv = pr[i];
+          bi = lane + 32 * i;
+        }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if (bi >= a.E) {  // a non-finite logit: flag it and keep the index valid
+        if (lane == 0) atomicExch(a.err, 2);
+        bi = k;
+        bv = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < kRoutePerLane; ++i)
+        if (lane + 32 * i == bi) pr[i] = -1.f;
+      if (lane == 0) {
+        a.sel[t * a.top_k + k] = bi;
+        a.wt[t * a.top_k + k] = bv;
+      }
+      wsum += bv;
+    }
+    __syncwarp();
+    if (lane < a.top_k) a.wt[t * a.top_k + lane] = wsum > 0.f ? a.wt[t * a.top_k + lane] / wsum : 0.f;
+  }
+  __syncthreads();
+  for (int e = warp; e < a.E; e += nw) {
+    int run = 0;
+    for (int i0 = 0; i0 < P; i0 += 32) {
+      const int i = i0 + lane;
+      const bool m = i < P && a.sel[i] == e;
+      const unsigned b = __ballot_sync(0xffffffffu, m);
+      if (m) rank[i] = run + __popc(b & ((1u << lane) - 1u));
+      run += __popc(b);
+    }
+    if (lane == 0) cnt[e] = run;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int o = 0;
+    for (int e = 0; e < a.E; ++e) {
+      off[e] = o;
+      a.range[2 * e] = o;
+      a.range[2 * e + 1] = cnt[e];
+      o += cnt[e];
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < P; i += kRouteThreads) {
+    const int row = off[a.sel[i]] + rank[i];
+    a.row_of[i] = row;
+    a.tok_of[row] = i / a.top_k;
+  }
+}
+
+// ghi/glo[r] = hi/lo[tok_of[r]] (rows of d fp16), one block per row
+__global__ void moe_gather_kernel(const int* tok_of, const __half* hi, const __half* lo, __half* ghi, __half* glo,
+                                  int d) {
+  const int r = blockIdx.x;
+  const size_t src = (size_t)tok_of[r] * d, dst = (size_t)r * d;
+  for (int i = threadIdx.x * 8; i < d; i += blockDim.x * 8) {
+    *reinterpret_cast<uint4*>(ghi + dst + i) = *reinterpret_cast<const uint4*>(hi + src + i);
+    *reinterpret_cast<uint4*>(glo + dst + i) = *reinterpret_cast<const uint4*>(lo + src + i);
+  }
+}
+
+// x[t] += sum_k wt[t][k] * y[row_of[t][k]], k in order; one block per token
+__global__ void moe_combine_kernel(const float* y, const int* row_of, const float* wt, float* x, int top_k, int d) {
+  const int t = blockIdx.x;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    float acc = 0.f;
+    for (int k = 0; k < top_k; ++k) acc = fmaf(wt[t * top_k + k], y[(size_t)row_of[t * top_k + k] * d + i], acc);
+    x[(size_t)t * d + i] += acc;
+  }
 }
 
 // ---------------------------------------------------------------- tensor-core attention
@@ -568,6 +704,33 @@ cudaError_t embed(const int* tok, const __half* E, float* x, int T, int d, cudaS
 cudaError_t rmsnorm_split(const float* x, const __half* g, __half* hi, __half* lo, int T, int d, float eps,
                           cudaStream_t st) {
   rmsnorm_split_kernel<<<T, 256, 0, st>>>(x, g, hi, lo, d, eps);
+  return cudaGetLastError();
+}
+
+cudaError_t moe_route(const RouteArgs& a, cudaStream_t st) {
+  const int smem = (a.T * a.top_k + 2 * a.E) * 4;
+  static bool attr[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(moe_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (kChunk * 8 + 2 * 256) * 4);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr[dev] = true;
+  }
+  moe_route_kernel<<<1, kRouteThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t moe_gather(const int* tok_of, const __half* hi, const __half* lo, __half* ghi, __half* glo, int rows,
+                       int d, cudaStream_t st) {
+  moe_gather_kernel<<<rows, 128, 0, st>>>(tok_of, hi, lo, ghi, glo, d);
+  return cudaGetLastError();
+}
+
+cudaError_t moe_combine(const float* y, const int* row_of, const float* wt, float* x, int T, int top_k, int d,
+                        cudaStream_t st) {
+  moe_combine_kernel<<<T, 256, 0, st>>>(y, row_of, wt, x, top_k, d);
   return cudaGetLastError();
 }
 

@@ -1,5 +1,6 @@
-// Chunked tensor-core prompt prefill (dense models): kernels and launchers of
-// prefill.cu, used by the host side of libkie. Internal, not part of the ABI.
+// Chunked tensor-core prompt prefill (dense and MoE models): kernels and
+// launchers of prefill.cu, used by the host side of libkie. Internal, not part
+// of the ABI.
 #pragma once
 
 #include <cuda.h>
@@ -19,7 +20,7 @@ constexpr int kGemmThreads = 128;
 constexpr int kGemmSmem = kStages * (kTileA + 2 * kTileB) + 1024 + 256;
 constexpr int kChunk = 1024;  // prompt tokens per chunk (activation buffers hold this many)
 
-enum Epi { EPI_QKV = 0, EPI_RESID = 1, EPI_SWIGLU = 2 };
+enum Epi { EPI_QKV = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_STORE = 3 };
 
 struct GemmArgs {
   int M, N, K;  // weight rows, tokens, input length
@@ -34,7 +35,28 @@ struct GemmArgs {
   // EPI_SWIGLU: rows gate_0, up_0, gate_1, ...; h[N][ff] = silu(gate) * up as fp16 hi/lo
   __half *h_hi, *h_lo;
   int ff;
+  // EPI_STORE: out[N][M] = D^T (fp32)
+  float* out;
+  // token rows taken from a device-resident range (one routed expert's rows
+  // of the expert-sorted activations): when nrange is set, the tokens are rows
+  // nrange[0] .. nrange[0] + nrange[1] - 1 of B and of the output (N is then
+  // only the grid's bound); tiles past the count exit at once
+  const int* nrange;
   int* err;  // set to 1 when a bounded wait gives up
+};
+
+// MoE routing of a chunk (the decode kernel's rule): per token, softmax
+// numerators of the router logits, the top_k by value with the lower expert
+// index on ties, weights renormalised over the chosen ones.
+struct RouteArgs {
+  const float* logits;  // [T][E]
+  int* sel;             // [T][top_k] chosen experts
+  float* wt;            // [T][top_k] their weights
+  int* range;           // [E][2]: row offset and count of each expert in the sorted pairs
+  int* row_of;          // [T][top_k]: the pair's row in the expert-sorted order
+  int* tok_of;          // [T * top_k]: the token of each sorted row
+  int* err;             // set to 2 on a non-finite router logit
+  int T, E, top_k;
 };
 
 struct AttnArgs {
@@ -55,6 +77,15 @@ cudaError_t rmsnorm_split(const float* x, const __half* g, __half* hi, __half* l
                           cudaStream_t st);
 // causal attention of a chunk over the cache on the tensor cores (mma.sync)
 cudaError_t attention(const AttnArgs& a, cudaStream_t st);
+// MoE: routing, the stable sort of (token, slot) pairs by expert, the gather of
+// the normalised rows in that order, and the weighted combine of the experts'
+// outputs into the residual stream (x[t] += sum_k wt[t][k] y[row_of[t][k]], k
+// in order)
+cudaError_t moe_route(const RouteArgs& a, cudaStream_t st);
+cudaError_t moe_gather(const int* tok_of, const __half* hi, const __half* lo, __half* ghi, __half* glo, int rows,
+                       int d, cudaStream_t st);
+cudaError_t moe_combine(const float* y, const int* row_of, const float* wt, float* x, int T, int top_k, int d,
+                        cudaStream_t st);
 
 }  // namespace pf
 }  // namespace kie
