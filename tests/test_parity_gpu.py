@@ -230,7 +230,10 @@ MOE_PROMPT_NS = S.Shape("moe-prompt-64x-top8-noshared", n_layers=2, d_model=512,
                         prompt_len=300, decode_len=16, max_ctx=316)
 
 
-@pytest.mark.parametrize("s", [S.SMALL, MOE_PROMPT, MOE_PROMPT_NS], ids=lambda s: s.name)
+MOE_PROMPT_2CHUNK = MOE_PROMPT_NS.with_(name="moe-prompt-2-chunks", prompt_len=1100, max_ctx=1116)
+
+
+@pytest.mark.parametrize("s", [S.SMALL, MOE_PROMPT, MOE_PROMPT_NS, MOE_PROMPT_2CHUNK], ids=lambda s: s.name)
 def test_prompt_path_matches_decode_path_and_oracle(s):
     # The tensor-core prompt path and the decode kernel run teacher-forced over
     # the same prompt fill caches whose next 16 steps agree with each other and
