@@ -405,7 +405,7 @@ def main():
         e2e = {"value": job_value(n * args.steps, ws, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(host_prompt.nbytes), "d2h_bytes_per_step": int(n * 4),
                "includes": f"reset + prefill of the {P}-token prompt from host memory + decode into pinned host memory"}
-        # the prompt path alone (tensor-core prefill for dense models)
+        # the prompt path alone (the tensor-core prefill)
         pms = []
         for _ in range(max(1, args.steps)):
             eng.reset()

@@ -405,8 +405,8 @@ kie_status make_plan(kie_ctx* c, const kie_config& k, int G, int sb, Plan& plan)
   return KIE_OK;
 }
 
-// The region cleared before every launch: control block, attention arrival
-// counters and the flagged scratch words (see Params).
+// The region cleared before every launch: control block and the flagged
+// scratch words (see Params).
 struct SyncLayout {
   size_t fx, fq, fo, fh, fcand, apart, froute, total;
 };
@@ -1418,8 +1418,8 @@ kie_status kie_decode(kie_ctx* c, int n, int32_t* out_tokens, const kie_decode_o
 //
 // kie_decode_static runs the same persistent decode kernel as kie_decode, but
 // the kernel's per-launch scratch (residual stream, q/k/v, attention output,
-// FFN hidden vector, attention partials and arrival counters, per-CTA argmax
-// candidates, control block) lives in this file-scope device array instead of
+// FFN hidden vector, attention chunk records, MoE router partials, per-CTA
+// argmax candidates, control block) lives in this file-scope device array instead of
 // buffers allocated with the context. The call itself allocates nothing.
 
 namespace {
@@ -1490,8 +1490,8 @@ extern "C" kie_status kie_decode_static(kie_ctx* c, int n, int32_t* out_tokens, 
   }
   cudaStream_t st = (cudaStream_t)stream;
   // the array keeps the previous call's contents: the barrier counter, the
-  // abort flag, the attention arrival counters and the flagged words' epochs
-  // must start at zero, which launch_on's clear of the sync region ensures
+  // abort flag and the flagged words' epochs must start at zero, which
+  // launch_on's clear of the sync region ensures
   const Run r{c->pending, n, 0, nullptr, out_tokens, nullptr, nullptr, 0, -1, -1, nullptr, 0};
   kie_status s = launch_on(c, r, base + lay.sync, lay.sync_bytes, st);
   if (s != KIE_OK) return s;
