@@ -106,12 +106,6 @@ struct kie_ctx {
   int *pf_sel = nullptr, *pf_range = nullptr, *pf_rowof = nullptr, *pf_tokof = nullptr;
   __half *pf_gh = nullptr, *pf_gl = nullptr, *pf_eh = nullptr, *pf_el = nullptr;
   std::vector<CUtensorMap> pf_emap;  // [L][E][2]
-  // tcgen05 attention: q as fp16 hi/lo parts, the transposed V copy (valid for
-  // positions 0 .. vt_valid - 1; the decode kernel does not write it, so a
-  // prompt call first transposes the positions decoded since) and the maps
-  __half *pf_qh = nullptr, *pf_ql = nullptr, *pf_vt = nullptr;
-  int pf_vt_ld = 0, pf_vt_valid = 0;
-  kie::pf::AttnMaps pf_amap{};
   std::vector<CUtensorMap> pf_rmap;  // [L]
   CUtensorMap pf_map_gh{}, pf_map_gl{}, pf_map_eh{}, pf_map_el{};
   float *pf_x = nullptr, *pf_q = nullptr;
@@ -510,17 +504,6 @@ static kie_status prefill_setup(kie_ctx* c) {
     CUDA_TRY(c, cudaMemset(c->pf_eh, 0, (size_t)rows * ffe * 2));
     CUDA_TRY(c, cudaMemset(c->pf_el, 0, (size_t)rows * ffe * 2));
   }
-  if (!c->pf_qh) {
-    c->pf_vt_ld = std::max(64, (k.max_ctx + 7) & ~7);
-    if ((s = dalloc(c, &c->pf_qh, (size_t)kChunk * hq * dh * 2)) ||
-        (s = dalloc(c, &c->pf_ql, (size_t)kChunk * hq * dh * 2)) ||
-        (s = dalloc(c, &c->pf_vt, (size_t)L * hk * dh * c->pf_vt_ld * 2)))
-      return s;
-    CUDA_TRY(c, cudaMemset(c->pf_qh, 0, (size_t)kChunk * hq * dh * 2));
-    CUDA_TRY(c, cudaMemset(c->pf_ql, 0, (size_t)kChunk * hq * dh * 2));
-    CUDA_TRY(c, cudaMemset(c->pf_vt, 0, (size_t)L * hk * dh * c->pf_vt_ld * 2));
-  }
-  c->pf_vt_valid = 0;
   if (!c->pf_x) {
     if ((s = dalloc(c, &c->pf_x, (size_t)kChunk * d * 4)) || (s = dalloc(c, &c->pf_q, (size_t)kChunk * hq * dh * 4)) ||
         (s = dalloc(c, &c->pf_xh, (size_t)kChunk * d * 2)) || (s = dalloc(c, &c->pf_xl, (size_t)kChunk * d * 2)) ||
@@ -568,10 +551,6 @@ static kie_status prefill_setup(kie_ctx* c) {
       }
     }
   }
-  ok = ok && make_map(&c->pf_amap.qh, c->pf_qh, kChunk, hq * dh, 128) &&
-       make_map(&c->pf_amap.ql, c->pf_ql, kChunk, hq * dh, 128) &&
-       make_map(&c->pf_amap.k, c->kcache, L * hk * k.max_ctx + 128, dh, 128) &&
-       make_map(&c->pf_amap.vt, c->pf_vt, L * hk * dh, c->pf_vt_ld, dh);
   if (!ok) return fail(c, KIE_ERR_CUDA, "tensor map encoding for the prefill failed");
   c->pf_ready = true;
   return KIE_OK;
@@ -588,8 +567,6 @@ static kie_status prefill_tc(kie_ctx* c, const std::vector<int32_t>& seq, cudaSt
   const int ff = moe ? k.ffn_shared : k.ffn, E = k.n_experts, ffe = k.ffn_expert, K = k.top_k;
   const int qkv_rows = (hq + 2 * hk) * dh;
   CUDA_TRY(c, cudaMemsetAsync(c->pf_err, 0, 4, st));
-  // the transposed V copy of the positions decoded since the last prompt call
-  CUDA_TRY(c, transpose_v(c->vcache, c->pf_vt, L, hk, dh, k.max_ctx, c->pf_vt_ld, c->pf_vt_valid, c->pos, st));
   for (size_t c0 = 0; c0 < seq.size(); c0 += kChunk) {
     const int T = (int)std::min<size_t>(kChunk, seq.size() - c0);
     const int p0 = c->pos + (int)c0;
@@ -602,13 +579,12 @@ static kie_status prefill_tc(kie_ctx* c, const std::vector<int32_t>& seq, cudaSt
       g.err = c->pf_err;
       g.M = qkv_rows; g.N = T; g.K = d; g.epi = EPI_QKV;
       g.q = c->pf_q; g.kcache = c->kcache; g.vcache = c->vcache; g.rope = c->rope;
-      g.q_hi = c->pf_qh; g.q_lo = c->pf_ql; g.vt = c->pf_vt; g.vt_ld = c->pf_vt_ld;
       g.layer = l; g.hq = hq; g.hk = hk; g.dh = dh; g.max_ctx = k.max_ctx; g.pos0 = p0;
       CUDA_TRY(c, gemm(W[0], c->pf_map_xh, c->pf_map_xl, g, st));
       c->launches += 2;
       if (l == L - 1) break;  // later positions need only this layer's K and V
-      AttnArgs at{c->pf_q, c->kcache, c->vcache, c->pf_oh, c->pf_ol, T, p0, l, hq, hk, dh, k.max_ctx, c->pf_err};
-      CUDA_TRY(c, attention_tc5(c->pf_amap, at, st));
+      AttnArgs at{c->pf_q, c->kcache, c->vcache, c->pf_oh, c->pf_ol, T, p0, l, hq, hk, dh, k.max_ctx};
+      CUDA_TRY(c, attention(at, st));
       GemmArgs o{};
       o.err = c->pf_err;
       o.M = d; o.N = T; o.K = hq * dh; o.epi = EPI_RESID; o.x = c->pf_x;
@@ -769,12 +745,7 @@ kie_status kie_create(const kie_config* cfg, int device, kie_ctx** out) {
 
   kie_status s;
   const size_t kv = (size_t)k.n_layers * hk * k.max_ctx * dh * sizeof(__half);
-  // the K cache has 128 rows of zero slack past its end: the prompt path's
-  // tensor map over it then always covers a whole 128-row box
-  const size_t k_slack = (size_t)128 * dh * sizeof(__half);
-  if ((s = dalloc(c, &c->kcache, kv + k_slack)) || (s = dalloc(c, &c->vcache, kv))) return bail(s);
-  if (cudaMemset(reinterpret_cast<unsigned char*>(c->kcache) + kv, 0, k_slack) != cudaSuccess)
-    return bail(fail(c, KIE_ERR_CUDA, "cudaMemset of the K cache slack failed"));
+  if ((s = dalloc(c, &c->kcache, kv)) || (s = dalloc(c, &c->vcache, kv))) return bail(s);
   if ((s = dalloc(c, &c->rope, (size_t)k.max_ctx * (dh / 2) * sizeof(float2)))) return bail(s);
   {
     std::vector<float2> tab((size_t)k.max_ctx * (dh / 2));
@@ -825,7 +796,6 @@ kie_status kie_reset(kie_ctx* c) {
   c->pos = 0;
   c->pending = -1;
   c->poisoned = false;
-  c->pf_vt_valid = 0;
   return KIE_OK;
 }
 
@@ -839,7 +809,6 @@ kie_status kie_rewind(kie_ctx* c, int32_t pos, int32_t pending) {
     return fail(c, KIE_ERR_INVALID_ARG, "pending token %d outside [0, %d)", pending, c->cfg.vocab);
   c->pos = pos;
   c->pending = pending;
-  c->pf_vt_valid = std::min(c->pf_vt_valid, pos);
   return KIE_OK;
 }
 
@@ -1205,7 +1174,6 @@ kie_status kie_load_weights(kie_ctx* c, const kie_tensor* tensors, int n, void* 
   c->pos = 0;
   c->pending = -1;
   c->poisoned = false;
-  c->pf_vt_valid = 0;
   return KIE_OK;
 }
 
@@ -1339,7 +1307,6 @@ kie_status kie_prefill(kie_ctx* c, const int32_t* tokens, int n, void* stream) {
     return s;
   }
   c->pos += (int32_t)seq.size();
-  c->pf_vt_valid = c->pos;  // the q/k/v epilogues wrote the transposed V of every prompt position
   c->pending = new_pending;
   return KIE_OK;
 }

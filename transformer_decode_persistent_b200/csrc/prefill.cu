@@ -169,14 +169,11 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, int row, int tb, int
       const float r = (vr & 1) ? (x0 * cs.y + x1 * cs.x) : (x0 * cs.x - x1 * cs.y);
       if (H < a.hq) {
         a.q[(size_t)t * a.hq * dh + (size_t)H * dh + dim] = r * scale;
-        if (a.q_hi) split_store(a.q_hi, a.q_lo, (size_t)t * a.hq * dh + (size_t)H * dh + dim, r * scale);
       } else {
         a.kcache[((size_t)(a.layer * a.hk + (H - a.hq)) * a.max_ctx + pos) * dh + dim] = __float2half_rn(r);
       }
     } else {
-      const __half hv = __float2half_rn(v[j]);
-      a.vcache[((size_t)(a.layer * a.hk + (H - a.hq - a.hk)) * a.max_ctx + pos) * dh + dim] = hv;
-      if (a.vt) a.vt[((size_t)(a.layer * a.hk + (H - a.hq - a.hk)) * dh + dim) * a.vt_ld + pos] = hv;
+      a.vcache[((size_t)(a.layer * a.hk + (H - a.hq - a.hk)) * a.max_ctx + pos) * dh + dim] = __float2half_rn(v[j]);
     }
   }
 }
@@ -278,7 +275,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kBN));
 }
-
 
 // ---------------------------------------------------------------- small kernels
 
@@ -676,265 +672,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 
 }  // namespace
 
-// ---------------------------------------------------------------- tcgen05 attention
-//
-// Causal attention of the chunk's queries over the cache with the
-// 5th-generation tensor cores. Block (query head h, 128 queries), 4 warps;
-// thread r owns query row r, which is tensor-memory lane r. Per block of 128
-// keys j: S = Q K_j^T (q as fp16 hi + lo parts, two MMAs per 16-wide K step,
-// fp32 accumulator in tensor memory); each thread reads its row of S, applies
-// the causal mask and the online softmax, rescales its row of O in tensor
-// memory when the running maximum grew, and writes its row of P (fp16) into
-// shared memory in the 128-byte-swizzled K-major layout the MMA reads; then
-// O += P V_j (V from the transposed copy, so that it is K-major over the keys).
-// K and V blocks are double-buffered by TMA. Q, K, V^T and P tiles are [rows x
-// 64 fp16] slices of 128-byte rows, 8-row groups 1024 bytes apart (the layout
-// TMA writes with 128-byte swizzle).
-template <int DH>
-struct Tc5 {
-  static constexpr int QS = DH / 64;                 // 64-wide slices of a head
-  static constexpr int kSlice = 128 * 128;           // [128 rows][64 fp16]
-  static constexpr int kVtSlice = DH * 128;          // [DH rows][64 fp16]
-  static constexpr int kQh = 0, kQl = QS * kSlice;
-  static constexpr int kK = 2 * QS * kSlice;         // [2 buffers][QS slices]
-  static constexpr int kVt = kK + 2 * QS * kSlice;   // [2 buffers][2 slices of 64 keys]
-  static constexpr int kP = kVt + 4 * kVtSlice;      // [2 slices of 64 keys]
-  static constexpr int kBar = kP + 2 * kSlice;
-  static constexpr int kSmem = kBar + 128 + 1024;    // barriers, tensor-memory address, alignment slack
-  static constexpr uint32_t kIdescPV = (1u << 4) | ((uint32_t)(DH >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
-};
-
-__device__ __forceinline__ void mma_id(uint32_t tmem, uint64_t a, uint64_t b, uint32_t idesc, bool acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"((unsigned)acc)
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
-  uint32_t r[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[i]);
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
-      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
-      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
-      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
-
-template <int DH>
-__global__ void __launch_bounds__(128, 1)
-    tc5_attention_kernel(const __grid_constant__ CUtensorMap tmQh, const __grid_constant__ CUtensorMap tmQl,
-                         const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmVt,
-                         const AttnArgs a) {
-  using C = Tc5<DH>;
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint64_t* kv_full = reinterpret_cast<uint64_t*>(smem + C::kBar);
-  uint64_t* kv_empty = kv_full + 2;
-  uint64_t* q_full = kv_empty + 2;
-  uint64_t* s_full = q_full + 1;
-  uint64_t* pv_done = s_full + 1;
-  uint32_t* taddr_s = reinterpret_cast<uint32_t*>(pv_done + 1);
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int qt = blockIdx.x, h = blockIdx.y;
-  const int g = (h * a.hk) / a.hq;
-  const int q0 = qt * 128;
-  const int qlast = min(a.T, q0 + 128) - 1;
-  const int last = a.pos0 + qlast;        // last key any row of the block sees
-  const int nblk = last / 128 + 1;
-  const int krow0 = (a.layer * a.hk + g) * a.max_ctx;
-  const int vrow0 = (a.layer * a.hk + g) * DH;
-  const int qrow = q0 + tid;
-  const int lim = qrow < a.T ? a.pos0 + qrow : last;  // last key of this row (rows past T: any finite)
-
-  if (tid == 0) {
-    for (int b = 0; b < 2; ++b) {
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(&kv_full[b])));
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(&kv_empty[b])));
-    }
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(q_full)));
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(s_full)));
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(pv_done)));
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(taddr_s)), "r"(256));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-  }
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-  __syncthreads();
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  const uint32_t tmem = *taddr_s;
-  const uint32_t tS = tmem, tO = tmem + 128;             // columns 0..127: S; 128..: O
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;  // this warp's tensor-memory lanes
-
-  auto load_kv = [&](int b, int j) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(&kv_full[b])),
-                 "r"(C::QS * C::kSlice + 2 * C::kVtSlice)
-                 : "memory");
-#pragma unroll
-    for (int sl = 0; sl < C::QS; ++sl)
-      tma2d(su32(smem + C::kK + (b * C::QS + sl) * C::kSlice), &tmK, sl * 64, krow0 + j * 128, su32(&kv_full[b]));
-#pragma unroll
-    for (int sl = 0; sl < 2; ++sl)
-      tma2d(su32(smem + C::kVt + (b * 2 + sl) * C::kVtSlice), &tmVt, j * 128 + sl * 64, vrow0, su32(&kv_full[b]));
-  };
-  if (tid == 0) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(q_full)), "r"(2 * C::QS * C::kSlice)
-                 : "memory");
-#pragma unroll
-    for (int sl = 0; sl < C::QS; ++sl) {
-      tma2d(su32(smem + C::kQh + sl * C::kSlice), &tmQh, h * DH + sl * 64, q0, su32(q_full));
-      tma2d(su32(smem + C::kQl + sl * C::kSlice), &tmQl, h * DH + sl * 64, q0, su32(q_full));
-    }
-    load_kv(0, 0);
-    if (nblk > 1) load_kv(1, 1);
-  }
-
-  float m = -INFINITY, l = 0.f;
-  for (int j = 0; j < nblk; ++j) {
-    const int b = j & 1;
-    if (tid == 32) {  // S = Q K_j^T
-      if (j == 0) mbar_wait(su32(q_full), 0u, a.err);
-      mbar_wait(su32(&kv_full[b]), (unsigned)(j >> 1) & 1u, a.err);
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-#pragma unroll
-      for (int sl = 0; sl < C::QS; ++sl) {
-        const uint64_t dqh = sdesc(su32(smem + C::kQh + sl * C::kSlice));
-        const uint64_t dql = sdesc(su32(smem + C::kQl + sl * C::kSlice));
-        const uint64_t dk = sdesc(su32(smem + C::kK + (b * C::QS + sl) * C::kSlice));
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          mma(tS, dqh + 2 * ks, dk + 2 * ks, sl > 0 || ks > 0);
-          mma(tS, dql + 2 * ks, dk + 2 * ks, true);
-        }
-      }
-      commit(su32(s_full));
-    }
-    mbar_wait(su32(s_full), (unsigned)j & 1u, a.err);
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    // row maximum over this block's valid keys
-    const int kbase = j * 128;
-    float mx = m;
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      float v[32];
-      tmem_ld32(tS + lane_off + (uint32_t)(c * 32), v);
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (kbase + c * 32 + i <= lim) mx = fmaxf(mx, v[i]);
-    }
-    const float alpha = (m == -INFINITY) ? 0.f : expf(m - mx);
-    // P and O are free once the previous block's P V is done
-    if (j > 0) {
-      mbar_wait(su32(pv_done), (unsigned)(j - 1) & 1u, a.err);
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      // tcgen05.ld/st are warp-collective (.sync.aligned): the warp rescales
-      // its rows together when any of them needs it (factor 1 leaves a row)
-      if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-        for (int c = 0; c < DH / 32; ++c) {
-          float v[32];
-          tmem_ld32(tO + lane_off + (uint32_t)(c * 32), v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= alpha;
-          tmem_st32(tO + lane_off + (uint32_t)(c * 32), v);
-        }
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-      }
-    }
-    float lsum = 0.f;
-    unsigned char* prow = smem + C::kP + (tid >> 3) * 1024 + (tid & 7) * 128;
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      float v[32];
-      tmem_ld32(tS + lane_off + (uint32_t)(c * 32), v);
-      uint32_t w[16];
-#pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        const float p0 = (kbase + c * 32 + i <= lim) ? expf(v[i] - mx) : 0.f;
-        const float p1 = (kbase + c * 32 + i + 1 <= lim) ? expf(v[i + 1] - mx) : 0.f;
-        lsum += p0 + p1;
-        w[i / 2] = pack_h2(p0, p1);
-      }
-      // keys 32c .. 32c+31: slice c/2, 16-byte chunks 4(c%2) .. 4(c%2)+3 of row tid
-      unsigned char* base = prow + (c >> 1) * C::kSlice;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int chunk = ((c & 1) * 4 + u) ^ (tid & 7);
-        *reinterpret_cast<uint4*>(base + chunk * 16) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-      }
-    }
-    l = l * alpha + lsum;
-    m = mx;
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // P writes before the MMA reads them
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    __syncthreads();
-    if (tid == 32) {  // O += P V_j
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-#pragma unroll
-      for (int sl = 0; sl < 2; ++sl) {
-        const uint64_t dp = sdesc(su32(smem + C::kP + sl * C::kSlice));
-        const uint64_t dv = sdesc(su32(smem + C::kVt + (b * 2 + sl) * C::kVtSlice));
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) mma_id(tO, dp + 2 * ks, dv + 2 * ks, C::kIdescPV, j > 0 || sl > 0 || ks > 0);
-      }
-      commit(su32(pv_done));
-      commit(su32(&kv_empty[b]));
-    }
-    if (tid == 0 && j + 2 < nblk) {
-      mbar_wait(su32(&kv_empty[b]), (unsigned)(j >> 1) & 1u, a.err);
-      load_kv(b, j + 2);
-    }
-  }
-  mbar_wait(su32(pv_done), (unsigned)(nblk - 1) & 1u, a.err);
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  const float inv = 1.0f / l;
-#pragma unroll 1
-  for (int c = 0; c < DH / 32; ++c) {
-    float v[32];
-    tmem_ld32(tO + lane_off + (uint32_t)(c * 32), v);
-    if (qrow < a.T) {
-      const size_t o = (size_t)qrow * a.hq * DH + (size_t)h * DH + c * 32;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) split_store(a.o_hi, a.o_lo, o + i, v[i] * inv);
-    }
-  }
-  // let the loads of blocks this CTA prefetched but never used land before exit
-  if (tid == 0) {
-    for (int j = max(nblk, 2) - 2; j < nblk; ++j)
-      if (j >= 0) mbar_wait(su32(&kv_full[j & 1]), (unsigned)(j >> 1) & 1u, a.err);
-  }
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-  __syncthreads();
-  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
-}
-
-// vt[((l hk + g) dh + i) vt_ld + p] = V[l][g][p][i]: one block per (l, g, 32
-// positions), a 32 x dh tile through shared memory
-__global__ void transpose_v_kernel(const __half* vcache, __half* vt, int hk, int dh, int max_ctx, int vt_ld, int p0,
-                                   int p1) {
-  __shared__ __half tile[32][128 + 2];
-  const int lg = blockIdx.y, pb = p0 + blockIdx.x * 32;
-  const __half* src = vcache + (size_t)lg * max_ctx * dh;
-  for (int i = threadIdx.x; i < 32 * dh; i += blockDim.x) {
-    const int r = i / dh, c = i - r * dh;
-    if (pb + r < p1) tile[r][c] = src[(size_t)(pb + r) * dh + c];
-  }
-  __syncthreads();
-  __half* dst = vt + (size_t)lg * dh * vt_ld;
-  for (int i = threadIdx.x; i < 32 * dh; i += blockDim.x) {
-    const int c = i / 32, r = i - c * 32;
-    if (pb + r < p1) dst[(size_t)c * vt_ld + pb + r] = tile[r][c];
-  }
-}
-
-
 bool make_map(CUtensorMap* map, const __half* base, int rows, int cols, int box_rows) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
   if (!enc) return false;
@@ -998,33 +735,6 @@ cudaError_t moe_gather(const int* tok_of, const __half* hi, const __half* lo, __
 cudaError_t moe_combine(const float* y, const int* row_of, const float* wt, float* x, int T, int top_k, int d,
                         cudaStream_t st) {
   moe_combine_kernel<<<T, 256, 0, st>>>(y, row_of, wt, x, top_k, d);
-  return cudaGetLastError();
-}
-
-cudaError_t attention_tc5(const AttnMaps& mp, const AttnArgs& a, cudaStream_t st) {
-  const dim3 grid((a.T + 127) / 128, a.hq);
-  static bool attr[64][2] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const int k = a.dh == 128 ? 1 : 0;
-  if (dev < 0 || dev >= 64 || !attr[dev][k]) {
-    cudaError_t e = k ? cudaFuncSetAttribute(tc5_attention_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             Tc5<128>::kSmem)
-                      : cudaFuncSetAttribute(tc5_attention_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             Tc5<64>::kSmem);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr[dev][k] = true;
-  }
-  if (k) tc5_attention_kernel<128><<<grid, 128, Tc5<128>::kSmem, st>>>(mp.qh, mp.ql, mp.k, mp.vt, a);
-  else tc5_attention_kernel<64><<<grid, 128, Tc5<64>::kSmem, st>>>(mp.qh, mp.ql, mp.k, mp.vt, a);
-  return cudaGetLastError();
-}
-
-cudaError_t transpose_v(const __half* vcache, __half* vt, int L, int hk, int dh, int max_ctx, int vt_ld, int p0,
-                        int p1, cudaStream_t st) {
-  if (p1 <= p0) return cudaSuccess;
-  const dim3 grid((p1 - p0 + 31) / 32, L * hk);
-  transpose_v_kernel<<<grid, 256, 0, st>>>(vcache, vt, hk, dh, max_ctx, vt_ld, p0, p1);
   return cudaGetLastError();
 }
 

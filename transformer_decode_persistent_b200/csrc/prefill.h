@@ -27,10 +27,7 @@ struct GemmArgs {
   int epi;
   // EPI_QKV: rows in the packed q/k/v order (head dims 0, dh/2, 1, dh/2+1, ...)
   float* q;                  // [N][hq * dh] rotated q, scaled by 1/sqrt(dh)
-  __half *q_hi, *q_lo;       // the same q as fp16 hi/lo parts (tcgen05 attention's A operand)
   __half *kcache, *vcache;   // [L][hk][max_ctx][dh]
-  __half* vt;                // V transposed: [L][hk][dh][vt_ld] (tcgen05 attention's B operand)
-  int vt_ld;
   const float2* rope;        // [max_ctx][dh/2] (cos, sin)
   int layer, hq, hk, dh, max_ctx, pos0;
   // EPI_RESID: x[N][M] += D^T
@@ -67,14 +64,6 @@ struct AttnArgs {
   const __half *kcache, *vcache;
   __half *o_hi, *o_lo;  // [T][hq * dh]
   int T, pos0, layer, hq, hk, dh, max_ctx;
-  int* err;  // tcgen05 attention: set to 1 when a bounded wait gives up
-};
-
-// Tensor maps of the tcgen05 attention: q hi/lo [kChunk][hq * dh], the K cache
-// as [L * hk * max_ctx][dh] and the transposed V copy as [L * hk * dh][vt_ld],
-// all with 64-column boxes of 128 rows (V: dh rows).
-struct AttnMaps {
-  CUtensorMap qh, ql, k, vt;
 };
 
 // 2-D fp16 tensor map [rows][cols] (row-major) with boxes of kBK columns x
@@ -88,12 +77,6 @@ cudaError_t rmsnorm_split(const float* x, const __half* g, __half* hi, __half* l
                           cudaStream_t st);
 // causal attention of a chunk over the cache on the tensor cores (mma.sync)
 cudaError_t attention(const AttnArgs& a, cudaStream_t st);
-// the same with tcgen05 (S and O in tensor memory); needs the q hi/lo parts
-// and the transposed V copy of every cached position
-cudaError_t attention_tc5(const AttnMaps& m, const AttnArgs& a, cudaStream_t st);
-// vt[((l hk + g) dh + i) vt_ld + p] = V[l][g][p][i] for positions p0 .. p1 - 1
-cudaError_t transpose_v(const __half* vcache, __half* vt, int L, int hk, int dh, int max_ctx, int vt_ld, int p0,
-                        int p1, cudaStream_t st);
 // MoE: routing, the stable sort of (token, slot) pairs by expert, the gather of
 // the normalised rows in that order, and the weighted combine of the experts'
 // outputs into the residual stream (x[t] += sum_k wt[t][k] y[row_of[t][k]], k
