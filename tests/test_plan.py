@@ -185,3 +185,28 @@ def test_plan_balances_the_tape_over_ctas(shape):
     starts = r["off"][:, 0].astype(np.int64)
     sizes = np.append(starts[1:], info["tape_bytes"]) - starts
     assert sizes.max() <= 1.03 * sizes.mean() and sizes.min() >= 0.97 * sizes.mean()
+
+
+def test_plan_accepts_wide_gqa_groups_and_rejects_what_the_attention_cannot_split():
+    """Up to 16 query heads per KV head are attended in equal sub-units of at
+    most 4 (8:1 Llama-3-70B-like, 7:1 Qwen-like layouts plan); more than 16, or
+    uneven groups that would leave a sub-unit without a head (25 query heads
+    over 2 KV heads: groups of 13 and 12 in sub-units of 4), are rejected."""
+    for hq, hk in ((32, 4), (64, 8), (28, 4), (14, 2)):
+        s = S.Shape(f"gqa-{hq}:{hk}", n_layers=1, d_model=hq * 64, n_heads=hq, n_kv_heads=hk, head_dim=64,
+                    ffn=1024, vocab=1000, max_ctx=64)
+        K.plan(s, 148, 13312)
+    for hq, hk in ((34, 2), (25, 2)):
+        s = S.Shape(f"gqa-{hq}:{hk}", n_layers=1, d_model=hq * 64, n_heads=hq, n_kv_heads=hk, head_dim=64,
+                    ffn=1024, vocab=1000, max_ctx=64)
+        with pytest.raises(K.KieError) as ei:
+            K.plan(s, 148, 13312)
+        assert ei.value.status == -1 and "query heads" in str(ei.value)
+
+
+def test_plan_moe_without_shared_expert():
+    """ffn_shared = 0 is a valid MoE shape; a negative or unaligned width is not."""
+    K.plan(MOE_NOSHARED, 148, 13312)
+    for bad in (-8, 12):
+        with pytest.raises(K.KieError):
+            K.plan(MOE_NOSHARED.with_(ffn_shared=bad), 148, 13312)
