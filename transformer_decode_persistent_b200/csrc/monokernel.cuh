@@ -424,7 +424,9 @@ static __device__ bool wait_bar(const Params& P, SmemCtl* sc, uint64_t* b, unsig
 
 // ---------------------------------------------------------------- attention plan
 // Attention work for one layer at position pos (T = pos + 1 keys): units are
-// (KV head g, chunk of `per` positions), unit u handled by CTA u % grid; each
+// (KV head g, chunk of `per` positions), unit u handled by CTA u % grid. The
+// chunk length is about T hk / grid rounded up to whole warp sub-ranges, and
+// is lengthened when that would leave a few units over for a second wave; each
 // of the kConsumerWarps warps of a unit takes pw = per / kConsumerWarps
 // positions as nsb sub-blocks of 32. The K and V rows of every sub-block are
 // streamed through the ring like weight tiles: per (unit, sub-block round) the
@@ -451,15 +453,24 @@ __device__ __forceinline__ AttnPlan attn_plan(int pos, int hk, int hq, int grid)
   a.T = pos + 1;
   int per = (int)(((long long)a.T * hk + grid - 1) / grid);
   per = ((max(per, kUnitMin) + kUnitMin - 1) / kUnitMin) * kUnitMin;
+  const int gmax = (hq + hk - 1) / hk;  // query heads of the largest group
+  a.sub = (gmax + kMaxHeadsPerGroup - 1) / kMaxHeadsPerGroup;
+  a.hs = (gmax + a.sub - 1) / a.sub;
+  // a unit count just past the grid would leave a few CTAs with two units and
+  // every layer waiting for them: then take the most chunks that fit one wave
+  // (longer units, none doubled)
+  const int upc = hk * a.sub;  // units per chunk
+  if (upc * ((a.T + per - 1) / per) > grid && grid >= upc) {
+    const int nmax = grid / upc;
+    per = (a.T + nmax - 1) / nmax;
+    per = ((per + kUnitMin - 1) / kUnitMin) * kUnitMin;
+  }
   a.per = per;
   a.pw = per / kConsumerWarps;
   a.nsb = a.pw / kAttnSub;
   a.nchk = (a.T + per - 1) / per;
   a.split = (hq > hk && hq * a.nchk <= grid) ? 1 : 0;
-  const int gmax = (hq + hk - 1) / hk;  // query heads of the largest group
-  a.sub = (gmax + kMaxHeadsPerGroup - 1) / kMaxHeadsPerGroup;
-  a.hs = (gmax + a.sub - 1) / a.sub;
-  a.units = (a.split ? hq : hk * a.sub) * a.nchk;
+  a.units = (a.split ? hq : upc) * a.nchk;
   return a;
 }
 // Unit u: KV head g, chunk ch, query heads h_lo .. h_lo + nh - 1. KV head g
