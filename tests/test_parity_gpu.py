@@ -153,6 +153,24 @@ def test_gqa_groups_wider_than_one_unit(s):
     check_tokens(gt, ol, s.name)
 
 
+GRID_SMALL = S.Shape("gqa-367:40-d112", n_layers=2, d_model=112, n_heads=367, n_kv_heads=40, head_dim=64,
+                     ffn=224, vocab=1000, prompt_len=600, decode_len=12, max_ctx=612)
+
+
+def test_more_attention_units_than_ctas():
+    # d_model 112 gives 112 CTAs, fewer than one chunk's attention units (40
+    # KV heads in groups of 9 and 10 query heads, each group as sub-units of
+    # 4, 4 and 1 or 2: 120 units per chunk), so the chunks cannot be fitted
+    # into one wave: at 600+ positions (3 chunks per head) every CTA runs 3 or
+    # 4 units in a row and publishes their chunk records before it merges the
+    # heads whose chunk 0 it holds
+    s = GRID_SMALL
+    w = S.make_weights(s, seed=12, cache=False)
+    gl, ol, gt, _ = forced_sequence_case(s, 12, s.decode_len, prompt_len=s.prompt_len, weights=w)
+    check_step_logits(gl, ol, s.name)
+    check_tokens(gt, ol, s.name)
+
+
 ZERO_DENSE = S.Shape("zero-dense", n_layers=2, d_model=512, n_heads=8, n_kv_heads=2, head_dim=64,
                      ffn=1024, vocab=3000, prompt_len=9, decode_len=12, max_ctx=24)
 ZERO_MOE = S.Shape("zero-moe", n_layers=2, d_model=512, n_heads=8, n_kv_heads=2, head_dim=64, ffn=0,
@@ -296,7 +314,7 @@ def test_long_context_32k_one_layer_oracle_parity():
     # cache comes from the prompt's projections (layer 0 needs no attention
     # output for them), then 8 teacher-forced steps at positions 32767..32774
     # compare logits with the engine's (tensor-core prompt path, then decode
-    # attention over ~32K positions in 19 chunks per head, more units than CTAs).
+    # attention over ~32K positions in 17 chunks per head: 136 units on 148 CTAs).
     s = S.LONG_2B.with_(name="gqa20:8-32k-1L", n_layers=1, decode_len=8, max_ctx=32768 + 8)
     w = S.make_weights(s, seed=4, cache=False)
     prompt = S.make_prompt(s, 4)
