@@ -196,6 +196,11 @@ def test_plan_accepts_wide_gqa_groups_and_rejects_what_the_attention_cannot_spli
         s = S.Shape(f"gqa-{hq}:{hk}", n_layers=1, d_model=hq * 64, n_heads=hq, n_kv_heads=hk, head_dim=64,
                     ffn=1024, vocab=1000, max_ctx=64)
         K.plan(s, 148, 13312)
+    # uneven groups of 9 and 10 query heads (sub-units of 4, 4 and 1 or 2) on a
+    # grid of 112 CTAs, fewer than one chunk's 120 attention units
+    s = S.Shape("gqa-367:40-d112", n_layers=1, d_model=112, n_heads=367, n_kv_heads=40, head_dim=64,
+                ffn=224, vocab=1000, max_ctx=612)
+    K.plan(s, 112, 13312)
     for hq, hk in ((34, 2), (25, 2)):
         s = S.Shape(f"gqa-{hq}:{hk}", n_layers=1, d_model=hq * 64, n_heads=hq, n_kv_heads=hk, head_dim=64,
                     ffn=1024, vocab=1000, max_ctx=64)
